@@ -1,0 +1,173 @@
+/*
+ * Prop2D CPU oracle: plain, single-threaded, fp64.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the correctness reference that the
+ * CUDA library is checked against.  Only the test suite, the package's
+ * smoke check and the CPU-baseline leg of the benchmark may load it.  It
+ * shares no code, header, table or constant with the CUDA path.
+ *
+ * What it computes (paper: "Scaling Parallel Sequence Models to
+ * Foundation-Scale Vision Encoders", Sec. 3 "Line-scan recurrence" and the
+ * papernotes.org summary of the method, "背景算子" paragraph, Eq. 2/3):
+ *
+ *   For each batch b, latent channel c and direction d in
+ *   {top->bottom, bottom->top, left->right, right->left}, the grid is swept
+ *   one line at a time.  Every position q of line l is updated in parallel
+ *   from the three positions q-1, q, q+1 of the previous line:
+ *
+ *       h_l(q) = sum_k w_l(q,k) * h_{l-1}(q+k-1) + lambda_l(q) * x_l(q),
+ *       h_{-1} = 0,
+ *
+ *   and the output is the gated sum over the directions that are enabled,
+ *
+ *       y = sum_d u_d (.) h_d                   (papernotes.org, Eq. y_c =
+ *                                                 Prop2D(x_c; u, lambda, w)).
+ *
+ *   The tridiagonal weights are row-stochastic (Sec. 3 "Stability and
+ *   connectivity"; papernotes.org normalisation formula):
+ *
+ *       s_k = sigmoid(wt_k)   for every slot k whose neighbour is on the grid,
+ *       S   = max(sum_k s_k, eps),                      (Sec. 5.1 "Fused CUDA
+ *       w_k = s_k / S.                                    normalization":
+ *                                                         sigmoid, local sum,
+ *                                                         clamp, divide)
+ *
+ * Readings taken where the pages are silent (the equation bodies of Sec. 3
+ * were lost from the page text):
+ *   - no skip term, h_{-1} = 0;
+ *   - off-grid neighbour slots get weight 0 and are left out of the sum;
+ *   - the clamp acts on the denominator, eps = 1e-6;
+ *   - lambda, u and the logits are separate per direction;
+ *   - slot k names the absolute orthogonal offset k-1 (-1 = up / left);
+ *   - with share_w the logit field has one channel, used by every channel.
+ *
+ * Layouts (all contiguous, row-major):
+ *   x      [B][Cc][H][W]
+ *   lambda [B][4][Cc][H][W]
+ *   u      [B][4][Cc][H][W]
+ *   wlogit [B][4][Cw][3][H][W],   Cw = share_w ? 1 : Cc
+ *   out    [B][Cc][H][W]
+ * Direction slot order: 0 top->bottom, 1 bottom->top, 2 left->right,
+ * 3 right->left; bit d of `dirs` enables slot d.
+ *
+ * Return value: 0 on success, 1 on a bad argument (nothing written).
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_EPS 1e-6
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/* Index of element (i, j) of plane `plane` in a [..][H][W] tensor. */
+static size_t at(size_t plane, int H, int W, int i, int j) {
+    return (plane * (size_t)H + (size_t)i) * (size_t)W + (size_t)j;
+}
+
+/* Row-stochastic weights of one position, following the normalisation
+ * formula: sigmoid of each on-grid slot, local sum, clamp, divide.
+ * `lg[k]` are the three logits, `valid[k]` says whether slot k's neighbour
+ * lies on the grid. */
+static void normalise(const double lg[3], const int valid[3], double w[3]) {
+    double s[3];
+    double sum = 0.0;
+    for (int k = 0; k < 3; ++k) {
+        s[k] = valid[k] ? sigmoid(lg[k]) : 0.0;
+        sum += s[k];
+    }
+    double denom = sum > ORACLE_EPS ? sum : ORACLE_EPS;
+    for (int k = 0; k < 3; ++k) w[k] = s[k] / denom;
+}
+
+/* Grid position (i, j) of line `line`, position `q` along it, for direction d. */
+static void position(int d, int line, int q, int *i, int *j) {
+    if (d < 2) { *i = line; *j = q; }      /* row lines: top->bottom / bottom->top */
+    else       { *i = q;    *j = line; }   /* column lines: left->right / right->left */
+}
+
+int oracle_prop2d_weights_f64(const double *wlogit, int B, int Cc, int H, int W,
+                              int share_w, double *w_out) {
+    if (!wlogit || !w_out || B < 0 || Cc < 0 || H < 0 || W < 0) return 1;
+    int Cw = share_w ? 1 : Cc;
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < 4; ++d)
+            for (int c = 0; c < Cw; ++c) {
+                size_t base = ((size_t)(b * 4 + d) * (size_t)Cw + (size_t)c) * 3;
+                for (int i = 0; i < H; ++i)
+                    for (int j = 0; j < W; ++j) {
+                        /* the orthogonal coordinate is j for row lines, i for column lines */
+                        int q = d < 2 ? j : i;
+                        int M = d < 2 ? W : H;
+                        double lg[3], w[3];
+                        int valid[3];
+                        for (int k = 0; k < 3; ++k) {
+                            valid[k] = (q + k - 1 >= 0) && (q + k - 1 < M);
+                            lg[k] = valid[k] ? wlogit[at(base + k, H, W, i, j)] : 0.0;
+                        }
+                        normalise(lg, valid, w);
+                        for (int k = 0; k < 3; ++k) w_out[at(base + k, H, W, i, j)] = w[k];
+                    }
+            }
+    return 0;
+}
+
+int oracle_prop2d_f64(const double *x, const double *lambda, const double *wlogit,
+                      const double *u, int B, int Cc, int H, int W, int dirs,
+                      int share_w, double *out) {
+    if (!x || !lambda || !wlogit || !u || !out) return 1;
+    if (B < 0 || Cc < 0 || H < 0 || W < 0) return 1;
+    if (dirs < 1 || dirs > 15) return 1;
+    int Cw = share_w ? 1 : Cc;
+    int maxM = H > W ? H : W;
+    double *hprev = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    double *hcur = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    if (!hprev || !hcur) { free(hprev); free(hcur); return 1; }
+
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < Cc; ++c) {
+            size_t xp = (size_t)b * (size_t)Cc + (size_t)c;      /* plane of x and out */
+            for (int i = 0; i < H; ++i)
+                for (int j = 0; j < W; ++j) out[at(xp, H, W, i, j)] = 0.0;
+
+            for (int d = 0; d < 4; ++d) {
+                if (!(dirs & (1 << d))) continue;
+                size_t gp = ((size_t)b * 4 + (size_t)d) * (size_t)Cc + (size_t)c;   /* lambda, u */
+                size_t wp = (((size_t)b * 4 + (size_t)d) * (size_t)Cw +
+                             (size_t)(share_w ? 0 : c)) * 3;                       /* logits */
+                int L = d < 2 ? H : W;      /* number of lines swept */
+                int M = d < 2 ? W : H;      /* positions per line */
+                for (int q = 0; q < M; ++q) hprev[q] = 0.0;
+
+                for (int step = 0; step < L; ++step) {
+                    /* even slots sweep forward, odd slots sweep backward */
+                    int line = (d % 2 == 0) ? step : L - 1 - step;
+                    for (int q = 0; q < M; ++q) {
+                        int i, j;
+                        position(d, line, q, &i, &j);
+                        double lg[3], w[3];
+                        int valid[3];
+                        for (int k = 0; k < 3; ++k) {
+                            valid[k] = (q + k - 1 >= 0) && (q + k - 1 < M);
+                            lg[k] = valid[k] ? wlogit[at(wp + k, H, W, i, j)] : 0.0;
+                        }
+                        normalise(lg, valid, w);
+                        double acc = 0.0;
+                        for (int k = 0; k < 3; ++k)
+                            if (valid[k]) acc += w[k] * hprev[q + k - 1];
+                        acc += lambda[at(gp, H, W, i, j)] * x[at(xp, H, W, i, j)];
+                        hcur[q] = acc;
+                    }
+                    for (int q = 0; q < M; ++q) {
+                        int i, j;
+                        position(d, line, q, &i, &j);
+                        out[at(xp, H, W, i, j)] += u[at(gp, H, W, i, j)] * hcur[q];
+                    }
+                    double *t = hprev; hprev = hcur; hcur = t;
+                }
+            }
+        }
+    free(hprev);
+    free(hcur);
+    return 0;
+}
