@@ -1,0 +1,380 @@
+"""Prop2D forward benchmark (one JSON line on rank 0).
+
+A step is one gspn_prop2d_fwd call over one batch of the workload (default:
+the C-GSPN 1K layer, B=32, Cc=64, 74x74, bf16 inputs, fp32 state, four
+directions, per-channel weights), inputs resident in HBM.  The metric is
+Prop2D forward GB/s of algorithmic traffic (x once; lambda, u and the three
+logits once per direction; y once), whole job over all ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1k]
+  python bench.py --impl reference ...   (the CPU oracle on host cores)
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (the
+planes are independent, so there is no collective on the data path); time
+is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from spatial_propagation_vision_b200.workloads import WORKLOADS, workload_inputs  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(bytes_per_rank: int, world: int, seconds: float) -> float:
+    """Whole-job GB/s: bytes processed by all ranks over the slowest rank's time."""
+    return bytes_per_rank * world / seconds / 1e9
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        deadline = time.time() + 5
+        while not self.samples and time.time() < deadline:
+            time.sleep(0.02)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ts, line in self.samples:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        inwin = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        use = inwin or rows[-3:]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for _, p in use if num(p[1]) is not None]
+        smax = [num(p[2]) for _, p in use if num(p[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, p in use for n, v in zip(names, p[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(inwin),
+                "power_w_max": max((num(p[3]) or 0.0) for _, p in use)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------
+
+def oracle_planes_seconds(inp64, planes):
+    import oracle
+    t0 = time.perf_counter()
+    for (b, c) in planes:
+        oracle.prop2d(inp64["x"][b:b + 1, c:c + 1], inp64["lam"][b:b + 1, :, c:c + 1],
+                      inp64["wlogit"][b:b + 1, :, c:c + 1] if inp64["wlogit"].shape[2] > 1
+                      else inp64["wlogit"][b:b + 1], inp64["u"][b:b + 1, :, c:c + 1])
+    return time.perf_counter() - t0
+
+
+def cpu_inputs_f64(w, seed=0, planes=None):
+    inp = workload_inputs(w, seed=seed)
+    return {k: v.double().numpy() for k, v in inp.items()}
+
+
+def cpu_oracle_baseline(w, budget_s=12.0, max_passes=3):
+    """The oracle as it stands, one host core, on whole passes over the
+    workload's planes (repeated until about budget_s)."""
+    inp = cpu_inputs_f64(w)
+    planes = [(b, c) for b in range(w.B) for c in range(w.Cc)]
+    per_plane = w.algorithmic_bytes() / len(planes)
+    done, secs = 0, 0.0
+    chunk = 64
+    t_start = time.perf_counter()
+    while done < max_passes * len(planes):
+        sel = [planes[(done + i) % len(planes)] for i in range(chunk)]
+        secs += oracle_planes_seconds(inp, sel)
+        done += chunk
+        if time.perf_counter() - t_start > budget_s:
+            break
+    return {"value": per_plane * done / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} planes ({done / len(planes):.2f} passes) of the {w.name} workload, "
+                      f"fp64 single-threaded C, {secs:.1f} s"}
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    inp = cpu_inputs_f64(w)
+    planes = [(b, c) for b in range(w.B) for c in range(w.Cc)]
+    per_plane = w.algorithmic_bytes() / len(planes)
+    n = args.ref_planes
+    k = 0
+
+    def step():
+        nonlocal k
+        sel = [planes[(k * n + i) % len(planes)] for i in range(n)]
+        k += 1
+        return oracle_planes_seconds(inp, sel)
+
+    for _ in range(args.warmup):
+        step()
+    secs = sum(step() for _ in range(args.steps))
+    value = per_plane * n * args.steps / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{n} planes of the {w.name} workload per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+METRIC = "Prop2D fwd GB/s (algorithmic HBM bytes / time); % of B200 HBM peak; ms/call"
+
+
+def config_of(w, world):
+    inbytes = w.algorithmic_bytes()
+    return {"workload": f"{w.name}: B={w.B} Cc={w.Cc} H={w.H} W={w.W} {w.dtype} inputs, fp32 state, "
+                        f"dirs={w.dirs}, share_w={w.share_w}",
+            "B": w.B, "Cc": w.Cc, "H": w.H, "W": w.W, "dirs": w.dirs, "share_w": w.share_w,
+            "algorithmic_bytes_per_step_per_gpu": inbytes,
+            "l2": ("inputs larger than L2, no flush" if inbytes > L2_BYTES
+                   else "L2 flushed (256 MiB write) between timed steps"),
+            "parallelism": f"replicas x{world} (independent planes, no collective)"}
+
+
+def run_ours(args, w):
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from spatial_propagation_vision_b200 import prop2d
+
+    inp_cpu = workload_inputs(w, seed=rank)
+    d = {k: v.to(dev) for k, v in inp_cpu.items()}
+    out = torch.empty_like(d["x"])
+    stream = torch.cuda.Stream(dev)
+    nbytes = w.algorithmic_bytes()
+    flush = None
+    if nbytes <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        prop2d.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=w.dirs,
+                          share_w=w.share_w, out=out, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            if flush is not None:
+                flush.fill_(1.0)
+            call()
+    torch.cuda.synchronize(dev)
+    info = prop2d.launch_info()
+
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark("t0")
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(1.0)
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        end.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark("t1")
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    sampler.stop()
+    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    region_ms = start.elapsed_time(end)
+    if flush is not None:
+        # the flush writes are not Prop2D work: time only the calls
+        step_ms = sum(kernel_ms) / args.steps
+    else:
+        step_ms = region_ms / args.steps
+    step_ms = max_over_ranks(step_ms, world, dev)
+    avg_kernel_ms = max_over_ranks(statistics.mean(kernel_ms), world, dev)
+
+    # end to end: host buffers -> device -> Prop2D -> host, through the C ABI
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    h = {k: v.pin_memory() for k, v in inp_cpu.items()}
+    h["out"] = torch.empty_like(inp_cpu["x"]).pin_memory()
+    dd = {k: torch.empty_like(v, device=dev) for k, v in h.items()}
+    prop2d.prop2d_fwd_host(h, dd, dirs=w.dirs, share_w=w.share_w, stream=stream)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        prop2d.prop2d_fwd_host(h, dd, dirs=w.dirs, share_w=w.share_w, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    h2d = sum(v.numel() * v.element_size() for k, v in inp_cpu.items())
+    d2h = h["out"].numel() * h["out"].element_size()
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = peaks()
+    achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
+    value = job_value(nbytes, world, step_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded)",
+        "config": config_of(w, world),
+        "hbm_frac_of_measured_peak": value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": args.traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "prop2d_fused_kernel", "avg_launch_ms": avg_kernel_ms},
+        "e2e": {"value": job_value(nbytes, world, e2e_ms * 1e-3), "unit": "GB/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "gspn_prop2d_fwd_host (pinned host buffers)"},
+        "gpu_launches": args.steps * info["launches"],
+        "launch": info,
+        "clocks": sampler.summary(),
+    }
+    if args.cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_oracle_baseline(w, budget_s=args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="1k", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--ref-planes", type=int, default=64, help="oracle planes per reference step")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel, if captured for "
+                         "the current build")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,138 @@
+/*
+ * gspn.h -- C ABI of the B200 (sm_100a) Prop2D library, libgspn.so.
+ *
+ * Prop2D is the four-direction line-scan spatial propagation of GSPN, run in
+ * the compressed latent channel space of C-GSPN ("Scaling Parallel Sequence
+ * Models to Foundation-Scale Vision Encoders": Sec. 3 "Line-scan recurrence",
+ * Sec. 5.1 "Latent-space 2D propagation" and "Fused CUDA normalization";
+ * papernotes.org summary, "背景算子" paragraph and the operator
+ * y_c = Prop2D(x_c; u, lambda, w)).  For every batch b, latent channel c and
+ * enabled direction d, the grid is swept one line at a time and every
+ * position q of line l is updated in parallel from three neighbours of the
+ * previous line:
+ *
+ *     h_l(q) = sum_{k=0..2} w_l(q,k) h_{l-1}(q+k-1) + lambda_l(q) x_l(q),  h_{-1} = 0
+ *     y      = sum_d u_d * h_d
+ *
+ * with row-stochastic weights made from logits by sigmoid, a sum over the
+ * on-grid neighbours, a clamp of that sum at 1e-6 and a divide (Sec. 5.1
+ * "Fused CUDA normalization"; papernotes.org normalisation formula).  Slot k
+ * names the absolute orthogonal offset k-1 (-1 = left for row lines, up for
+ * column lines); off-grid slots carry no weight.  The normalisation is fused
+ * into the scan: the weights are never written anywhere.
+ *
+ * Layouts (element offsets, contiguous, row-major):
+ *   x      [B][Cc][H][W]
+ *   lambda [B][4][Cc][H][W]
+ *   u      [B][4][Cc][H][W]
+ *   wlogit [B][4][Cw][3][H][W]      Cw = share_w ? 1 : Cc
+ *   out    [B][Cc][H][W]
+ * Direction slots: 0 top->bottom, 1 bottom->top, 2 left->right,
+ * 3 right->left.  All four slots are always present in lambda, u and wlogit;
+ * slots not enabled by `dirs` are never read.
+ *
+ * Dtypes: inputs and output share one dtype (fp32 or bf16); the recurrence
+ * state, the weights and the direction sum are fp32.
+ *
+ * Ownership: the caller owns every buffer.  The library keeps no state
+ * between calls and allocates no memory.
+ *
+ * Errors: every entry point returns a gspn_status and never aborts or traps.
+ * Argument errors are detected on the host before anything is launched;
+ * a launch failure is reported as GSPN_ERR_CUDA (cudaGetLastError).
+ */
+#ifndef GSPN_H_
+#define GSPN_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GSPN_F32 = 0,   /* float32 inputs and output */
+    GSPN_BF16 = 1   /* bfloat16 inputs and output (fp32 state) */
+} gspn_dtype;
+
+typedef enum {
+    GSPN_OK = 0,
+    GSPN_ERR_NULL = 1,     /* a required pointer is NULL */
+    GSPN_ERR_SHAPE = 2,    /* B, Cc, H or W negative, or a size the library cannot index */
+    GSPN_ERR_DIRS = 3,     /* dirs outside 1..15, or share_w not 0/1 */
+    GSPN_ERR_DTYPE = 4,    /* unknown gspn_dtype */
+    GSPN_ERR_ALIGN = 5,    /* a device pointer is not 16-byte aligned */
+    GSPN_ERR_CUDA = 6,     /* the CUDA runtime reported an error */
+    GSPN_ERR_DEVICE = 7    /* the current device is not sm_100 (B200) */
+} gspn_status;
+
+enum {
+    GSPN_DIR_TB = 1,    /* top -> bottom: rows i = 0..H-1, previous row i-1 */
+    GSPN_DIR_BT = 2,    /* bottom -> top: rows i = H-1..0, previous row i+1 */
+    GSPN_DIR_LR = 4,    /* left -> right: columns j = 0..W-1, previous column j-1 */
+    GSPN_DIR_RL = 8,    /* right -> left: columns j = W-1..0, previous column j+1 */
+    GSPN_DIR_ALL = 15
+};
+
+/*
+ * gspn_prop2d_fwd -- y = Prop2D(x; u, lambda, w), forward.
+ *
+ * x, lambda, wlogit, u : device pointers, layouts above, dtype `dtype`,
+ *                        16-byte aligned.  Read only.
+ * B, Cc, H, W          : sizes, >= 0.  Any size is zero -> nothing to do, GSPN_OK.
+ * dirs                 : bitmask of GSPN_DIR_*, 1..15.
+ * share_w              : 0 -> one logit field per channel;
+ *                        1 -> one logit field per (batch, direction), used by
+ *                             every channel (the compact multi-channel mode of
+ *                             Sec. 4.2 "Channel-shared weights").
+ * dtype                : GSPN_F32 or GSPN_BF16.
+ * out                  : device pointer [B][Cc][H][W], dtype `dtype`, 16-byte
+ *                        aligned; fully overwritten.  Must not alias an input.
+ * stream               : CUDA stream; the call is asynchronous on it and does
+ *                        not synchronise.
+ *
+ * Returns GSPN_OK or the first error found; on an argument error nothing is
+ * launched and `out` is untouched.
+ */
+gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const void *wlogit,
+                            const void *u, int B, int Cc, int H, int W, int dirs,
+                            int share_w, gspn_dtype dtype, void *out,
+                            cudaStream_t stream);
+
+/*
+ * gspn_prop2d_fwd_host -- the same operation on HOST buffers.
+ *
+ * Copies the four host inputs (h_x, h_lambda, h_wlogit, h_u) into the
+ * caller's device buffers (d_x, d_lambda, d_wlogit, d_u) with
+ * cudaMemcpyAsync on `stream`, runs gspn_prop2d_fwd into d_out, copies d_out
+ * back into h_out, and synchronises `stream` before returning, so h_out is
+ * valid on return.  Host buffers should be pinned (page-locked) for the
+ * copies to run at full speed; pageable memory works but is slower.  Device
+ * buffers follow the rules of gspn_prop2d_fwd.  Nothing is allocated.
+ */
+gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda, const void *h_wlogit,
+                                 const void *h_u, void *h_out,
+                                 void *d_x, void *d_lambda, void *d_wlogit, void *d_u,
+                                 void *d_out,
+                                 int B, int Cc, int H, int W, int dirs, int share_w,
+                                 gspn_dtype dtype, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *gspn_status_str(gspn_status status);
+
+/*
+ * gspn_last_launch_info -- describes the kernel launches made by the last
+ * successful gspn_prop2d_fwd on the calling host thread: number of kernel
+ * launches, grid size, threads per block and dynamic shared memory bytes of
+ * the main kernel, and a short name of the path taken.  For diagnostics and
+ * benchmarks; any pointer may be NULL.
+ */
+void gspn_last_launch_info(int *launches, int *grid, int *block, int *smem_bytes,
+                           const char **path);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSPN_H_ */

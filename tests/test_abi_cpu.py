@@ -1,0 +1,76 @@
+"""The C ABI without a GPU: the library builds and loads, exports every
+function that include/gspn.h declares, and rejects bad arguments on the host
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from spatial_propagation_vision_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = build.build_library()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(gspn_[a-z0-9_]+)\s*\(",
+                                src, flags=re.M)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    assert "gspn_prop2d_fwd" in names and "gspn_status_str" in names, names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def _fwd(lib):
+    f = lib.gspn_prop2d_fwd
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 7 + [ctypes.c_void_p] * 2
+    f.restype = ctypes.c_int
+    return f
+
+
+P = 0x10000  # fake, 16-byte aligned "device" address: never dereferenced on these paths
+
+
+@pytest.mark.parametrize("args,status", [
+    ((P, P, P, P, -1, 4, 8, 8, 15, 0, 0, P), 2),          # negative B
+    ((P, P, P, P, 1, 4, 8, -8, 15, 0, 0, P), 2),          # negative W
+    ((P, P, P, P, 1, 4, 8, 8, 0, 0, 0, P), 3),            # empty direction mask
+    ((P, P, P, P, 1, 4, 8, 8, 16, 0, 0, P), 3),           # mask beyond the 4 directions
+    ((P, P, P, P, 1, 4, 8, 8, 15, 2, 0, P), 3),           # share_w not 0/1
+    ((P, P, P, P, 1, 4, 8, 8, 15, 0, 7, P), 4),           # unknown dtype
+    ((None, P, P, P, 1, 4, 8, 8, 15, 0, 0, P), 1),        # NULL input
+    ((P, P, P, P, 1, 4, 8, 8, 15, 0, 1, None), 1),        # NULL output
+    ((P + 2, P, P, P, 1, 4, 8, 8, 15, 0, 1, P), 5),       # misaligned input
+    ((P, P, P, P, 1, 4, 8, 8, 15, 0, 0, P + 4), 5),       # misaligned output
+    ((None, None, None, None, 0, 4, 8, 8, 15, 0, 0, None), 0),   # empty batch: nothing to do
+    ((None, None, None, None, 1, 4, 0, 8, 15, 0, 1, None), 0),   # empty grid
+    ((P, P, P, P, 1, 4, 8, 5000, 15, 0, 0, P), 2),        # line longer than any kernel takes
+])
+def test_argument_checks(lib, args, status):
+    assert _fwd(lib)(*args, None) == status
+
+
+def test_status_strings(lib):
+    lib.gspn_status_str.argtypes = [ctypes.c_int]
+    lib.gspn_status_str.restype = ctypes.c_char_p
+    for s in range(8):
+        assert lib.gspn_status_str(s).decode().startswith("GSPN_")
+    assert lib.gspn_status_str(99) is not None
