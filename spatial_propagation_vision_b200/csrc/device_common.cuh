@@ -49,6 +49,56 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// bulk (TMA engine, non-tensor) copies global -> shared completed on an
+// mbarrier, and the mbarrier operations around them.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(mbar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}" : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Set by a kernel whose bounded wait for an asynchronous copy gave up (the
+// copy never completed); read and cleared by gspn_device_status().  The
+// library is one translation unit, so this is its only definition.
+__device__ unsigned int g_gspn_device_status = 0;
+constexpr unsigned int kStatusCopyTimeout = 1u;
+constexpr long long kMaxWaitPolls = 1LL << 26;
+
+// Wait for phase `parity` of an mbarrier, polling at most kMaxWaitPolls
+// times; on timeout record it and return false (the caller carries on
+// with whatever the buffer holds, so the launch still terminates).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity) {
+    for (long long i = 0; i < kMaxWaitPolls; ++i)
+        if (mbar_try_wait(mbar, parity)) return true;
+    atomicOr(&g_gspn_device_status, kStatusCopyTimeout);
+    return false;
+}
+
+__device__ __forceinline__ void red_add_shared_if(uint32_t addr, float v, bool pred) {
+    asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p red.shared.add.f32 [%0], %1;\n}"
+                 ::"r"(addr), "f"(v), "r"(static_cast<uint32_t>(pred)) : "memory");
+}
+
 // Copy the 4-byte words [w0, w0 + nwords) of a global buffer to shared
 // memory, one warp cooperating.  `gsrc` is 4-byte aligned; `sdst` is the
 // shared address that receives gsrc's first byte and has the same address

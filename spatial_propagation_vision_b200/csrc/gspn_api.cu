@@ -8,13 +8,13 @@
 #include <mutex>
 
 #include "gspn.h"
-#include "prop2d_fused.cuh"
 #include "prop2d_generic.cuh"
+#include "prop2d_pair.cuh"
 
 namespace {
 
-using gspn::FusedParams;
 using gspn::GenericParams;
+using gspn::PairParams;
 
 struct LaunchInfo {
     int launches = 0, grid = 0, block = 0, smem = 0;
@@ -22,7 +22,7 @@ struct LaunchInfo {
 };
 thread_local LaunchInfo g_last;
 
-constexpr int kMaxFusedLine = 256;      // longest line (H or W) the fused kernel holds in registers
+constexpr int kMaxPairLine = 256;       // longest line (H or W) the paired kernel holds in registers
 constexpr int kMaxGenericLine = 4096;   // longest line the general kernel accepts
 
 struct DeviceProps {
@@ -49,110 +49,99 @@ cudaError_t device_props(DeviceProps &dp) {
 
 inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
-// Launch geometry of the fused kernel.
-struct FusedPlan {
-    bool ok = false;
+// Launch geometry of the paired-direction kernel.
+struct PairPlan {
     bool y_global = false;
     int smem = 0;
-    FusedParams p{};
+    PairParams p{};
 };
 
-// Shared-memory bytes of one tensor slot for the row directions.
-int row_slot_bytes(int t_row, int W, int es) { return round_up(t_row * W * es + 16, 16); }
-// ... and for the column directions (rows of pw words, one extra word every 32 rows).
-int col_slot_bytes(int H, int pw, int R) {
-    return round_up((H * pw + ((R % 2 == 0) ? H / 32 + 1 : 0)) * 4, 16);
+// Bytes of one (half, tensor) slot of the column ring (see ColLayout).
+int col_slot_bytes(int H, int R) {
+    const int words = (R % 2) ? H * 4 : H * 5 + 32;
+    return round_up(words * 4, 16);
 }
 
-// Choose chunk sizes and the output mode so that the CTA fits `cap` bytes.
-bool plan_fused_fit(FusedPlan &pl, int cap, int H, int W, int dirs, int es, int R,
-                    bool allow_yg, int min_seg_bytes) {
-    const bool any_row = dirs & 3, any_col = dirs & 12;
-    const int n_row = ((dirs & 1) ? 1 : 0) + ((dirs & 2) ? 1 : 0);
-    const int n_col = ((dirs & 4) ? 1 : 0) + ((dirs & 8) ? 1 : 0);
+// Choose the row chunk and the output mode so that one CTA fits `cap` bytes
+// of shared memory.  Output modes: the fp32 output plane in shared memory;
+// fp32 outputs accumulated in global memory (L2 atomics); row bands of the
+// output plane in shared memory (the scans are rerun per band).
+bool plan_pair_fit(PairPlan &pl, int cap, int H, int W, int dirs, int es, int R, bool allow_yg,
+                   int min_t_row) {
+    const bool row_on = dirs & 3, col_on = dirs & 12;
     const int YP = W | 1;
-    // output mode: full plane in smem, else (fp32) global atomics, else bands
+    const int slot_col = col_slot_bytes(H, R);
+    const int col_ring = col_on ? gspn::kColStages * 2 * gspn::kPairTensors * slot_col : 0;
+    // mbarriers of the row ring and the shift table of its staged spans, then
+    // a tail that keeps reads of positions past the end of a line in bounds
+    // (256 bytes: 3 mbarriers at 0, shift table at 64, 12 source pointers at 128)
+    const int pad = 256 + round_up(32 * R * 20 + 64, 16);
     for (int mode = 0; mode < 3; ++mode) {
         if (mode == 1 && !allow_yg) continue;
-        for (int seg_words = 8; seg_words >= 1; seg_words >>= 1) {
-            const int t_col = seg_words * 4 / es;
-            if (seg_words * 4 < min_seg_bytes) break;
-            if (es == 2 && (t_col % 2)) continue;
-            const int pw = (seg_words % 2 == 0) ? seg_words + 1 : seg_words;
-            const int slot_col = col_slot_bytes(H, pw, R);
-            const int col_ring = any_col ? n_col * gspn::kStages * gspn::kTensors * slot_col : 0;
-            for (int t_row = 8; t_row >= 1; t_row >>= 1) {
-                const int slot_row = row_slot_bytes(t_row, W, es);
-                const int row_ring = any_row ? n_row * gspn::kStages * gspn::kTensors * slot_row : 0;
-                int rings = col_ring + row_ring;
-                int band_rows = H, y_bytes = 0;
-                if (mode == 0) {
-                    y_bytes = round_up(H * YP * 4, 16);
-                } else if (mode == 2) {
-                    const int avail = cap - rings;
-                    if (avail < YP * 4) continue;
-                    band_rows = avail / (YP * 4);
-                    if (band_rows >= H) band_rows = H;
-                    y_bytes = round_up(band_rows * YP * 4, 16);
-                }
-                if (y_bytes + rings > cap) continue;
-                FusedParams &p = pl.p;
-                p.t_row = t_row;
-                p.slot_row = slot_row;
-                p.t_col = t_col;
-                p.words_col = seg_words;
-                p.pw_col = pw;
-                p.slot_col = slot_col;
-                p.y_pitch = YP;
-                p.band_rows = band_rows;
-                p.bands = (H + band_rows - 1) / band_rows;
-                int off = y_bytes;
-                for (int d = 0; d < 4; ++d) {
-                    if (!(dirs & (1 << d))) { p.ring_off[d] = -1; continue; }
-                    p.ring_off[d] = off;
-                    off += gspn::kStages * gspn::kTensors * (d < 2 ? slot_row : slot_col);
-                }
-                pl.smem = off;
-                pl.y_global = (mode == 1);
-                pl.ok = true;
-                return true;
+        for (int t_row = 8; t_row >= min_t_row; t_row >>= 1) {
+            // a staged span starts at its source address modulo 16 and is rounded up to 16 bytes
+            const int slot_row = round_up(t_row * W * es + 32, 16);
+            const int row_ring = row_on ? gspn::kRowStages * 2 * gspn::kPairTensors * slot_row : 0;
+            const int rings = row_ring + col_ring + pad;
+            int band_rows = H, y_bytes = 0;
+            if (mode == 0) {
+                y_bytes = round_up(H * YP * 4, 16);
+            } else if (mode == 2) {
+                if (cap - rings < YP * 4) continue;
+                band_rows = (cap - rings) / (YP * 4);
+                if (band_rows > H) band_rows = H;
+                y_bytes = round_up(band_rows * YP * 4, 16);
             }
+            if (y_bytes + rings > cap) continue;
+            PairParams &p = pl.p;
+            p.t_row = t_row;
+            p.slot_row = slot_row;
+            p.slot_col = slot_col;
+            p.ring_row = y_bytes;
+            p.ring_col = y_bytes + row_ring;
+            p.bar_off = y_bytes + row_ring + col_ring;
+            p.y_pitch = YP;
+            p.band_rows = band_rows;
+            p.bands = (H + band_rows - 1) / band_rows;
+            pl.smem = y_bytes + rings;
+            pl.y_global = mode == 1;
+            return true;
         }
     }
     return false;
 }
 
-template <typename T, int R, bool YG>
-cudaError_t launch_fused_t(const FusedPlan &pl, const DeviceProps &dp, cudaStream_t stream) {
-    auto kern = gspn::prop2d_fused_kernel<T, R, YG>;
+template <typename T, int R, int MODE>
+cudaError_t launch_pair_t(const PairPlan &pl, const DeviceProps &dp, cudaStream_t stream) {
+    auto kern = gspn::prop2d_pair_kernel<T, R, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kFusedThreads, pl.smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kPairThreads, pl.smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = static_cast<long long>(dp.sms) * per_sm;
     if (grid > pl.p.n_items) grid = pl.p.n_items;
-    kern<<<static_cast<unsigned>(grid), gspn::kFusedThreads, pl.smem, stream>>>(pl.p);
+    kern<<<static_cast<unsigned>(grid), gspn::kPairThreads, pl.smem, stream>>>(pl.p);
     g_last.launches = 1;
     g_last.grid = static_cast<int>(grid);
-    g_last.block = gspn::kFusedThreads;
+    g_last.block = gspn::kPairThreads;
     g_last.smem = pl.smem;
-    g_last.path = YG ? "fused-yglobal" : (pl.p.bands > 1 ? "fused-banded" : "fused");
+    g_last.path = MODE == gspn::kYGlobal ? "pair-yglobal" : MODE == gspn::kYBanded ? "pair-banded" : "pair";
     return cudaGetLastError();
 }
 
-template <typename T, bool YG>
-cudaError_t launch_fused_r(int R, const FusedPlan &pl, const DeviceProps &dp, cudaStream_t s) {
+template <typename T, int MODE>
+cudaError_t launch_pair_r(int R, const PairPlan &pl, const DeviceProps &dp, cudaStream_t s) {
     switch (R) {
-        case 1: return launch_fused_t<T, 1, YG>(pl, dp, s);
-        case 2: return launch_fused_t<T, 2, YG>(pl, dp, s);
-        case 3: return launch_fused_t<T, 3, YG>(pl, dp, s);
-        case 4: return launch_fused_t<T, 4, YG>(pl, dp, s);
-        case 5: return launch_fused_t<T, 5, YG>(pl, dp, s);
-        case 6: return launch_fused_t<T, 6, YG>(pl, dp, s);
-        case 7: return launch_fused_t<T, 7, YG>(pl, dp, s);
-        case 8: return launch_fused_t<T, 8, YG>(pl, dp, s);
+        case 1: return launch_pair_t<T, 1, MODE>(pl, dp, s);
+        case 2: return launch_pair_t<T, 2, MODE>(pl, dp, s);
+        case 3: return launch_pair_t<T, 3, MODE>(pl, dp, s);
+        case 4: return launch_pair_t<T, 4, MODE>(pl, dp, s);
+        case 5: return launch_pair_t<T, 5, MODE>(pl, dp, s);
+        case 6: return launch_pair_t<T, 6, MODE>(pl, dp, s);
+        case 7: return launch_pair_t<T, 7, MODE>(pl, dp, s);
+        case 8: return launch_pair_t<T, 8, MODE>(pl, dp, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -178,15 +167,15 @@ cudaError_t launch_generic(const GenericParams &gp0, const DeviceProps &dp, cuda
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kFusedThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kGenericThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = static_cast<long long>(dp.sms) * per_sm;
     if (grid > gp.n_items) grid = gp.n_items;
-    kern<<<static_cast<unsigned>(grid), gspn::kFusedThreads, smem, stream>>>(gp);
+    kern<<<static_cast<unsigned>(grid), gspn::kGenericThreads, smem, stream>>>(gp);
     g_last.launches = 1;
     g_last.grid = static_cast<int>(grid);
-    g_last.block = gspn::kFusedThreads;
+    g_last.block = gspn::kGenericThreads;
     g_last.smem = smem;
     g_last.path = "generic";
     return cudaGetLastError();
@@ -195,6 +184,18 @@ cudaError_t launch_generic(const GenericParams &gp0, const DeviceProps &dp, cuda
 bool misaligned(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) != 0; }
 
 }  // namespace
+
+extern "C" gspn_status gspn_device_status(unsigned int *flags, int clear) {
+    if (!flags) return GSPN_ERR_NULL;
+    if (cudaMemcpyFromSymbol(flags, gspn::g_gspn_device_status, sizeof(unsigned int)) != cudaSuccess)
+        return GSPN_ERR_CUDA;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(gspn::g_gspn_device_status, &zero, sizeof(unsigned int)) != cudaSuccess)
+            return GSPN_ERR_CUDA;
+    }
+    return GSPN_OK;
+}
 
 extern "C" const char *gspn_status_str(gspn_status s) {
     switch (s) {
@@ -245,25 +246,34 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
 
     const int es = dtype == GSPN_BF16 ? 2 : 4;
     cudaError_t err = cudaSuccess;
-    const bool fused_ok = maxline <= kMaxFusedLine && (es == 4 || (W % 2 == 0));
-    if (fused_ok) {
+    const bool pair_ok = maxline <= kMaxPairLine && H >= 2 && W >= 2 && (es == 4 || (W % 2 == 0));
+    if (pair_ok) {
         const int R = (maxline + 31) / 32;
-        FusedPlan pl;
+        PairPlan pl;
         pl.p.x = x; pl.p.lam = lambda; pl.p.wl = wlogit; pl.p.u = u; pl.p.out = out;
         pl.p.B = B; pl.p.Cc = Cc; pl.p.H = H; pl.p.W = W; pl.p.dirs = dirs; pl.p.share_w = share_w;
-        // Prefer two CTAs per SM with >= 16-byte column segments; then one CTA per SM.
-        const int cap2 = dp.smem_per_sm / 2 - 1024;
-        const int cap1 = dp.smem_optin;
-        bool fit = plan_fused_fit(pl, cap2 < cap1 ? cap2 : cap1, H, W, dirs, es, R, es == 4, 16) ||
-                   plan_fused_fit(pl, cap1, H, W, dirs, es, R, es == 4, 16) ||
-                   plan_fused_fit(pl, cap1, H, W, dirs, es, R, es == 4, 4);
+        // Prefer three CTAs per SM, then two, then one; bands only as a last resort.
+        const int caps[3] = {dp.smem_per_sm / 3 - 1024, dp.smem_per_sm / 2 - 1024, dp.smem_optin};
+        bool fit = false;
+        for (int ci = 0; ci < 3 && !fit; ++ci) {
+            const int cap = caps[ci] < dp.smem_optin ? caps[ci] : dp.smem_optin;
+            fit = plan_pair_fit(pl, cap, H, W, dirs, es, R, es == 4, 2);
+        }
+        if (!fit) fit = plan_pair_fit(pl, dp.smem_optin, H, W, dirs, es, R, es == 4, 1);
         if (fit) {
             pl.p.n_items = B * Cc * pl.p.bands;
+            const unsigned long long plane_bytes = static_cast<unsigned long long>(HW) * es;
+            pl.p.end_x = static_cast<unsigned long long>(B) * Cc * plane_bytes;
+            pl.p.end_gate = 4ULL * pl.p.end_x;
+            pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane_bytes;
+            const bool banded = pl.p.bands > 1;
             if (es == 4) {
-                err = pl.y_global ? launch_fused_r<float, true>(R, pl, dp, stream)
-                                  : launch_fused_r<float, false>(R, pl, dp, stream);
+                err = pl.y_global ? launch_pair_r<float, gspn::kYGlobal>(R, pl, dp, stream)
+                      : banded    ? launch_pair_r<float, gspn::kYBanded>(R, pl, dp, stream)
+                                  : launch_pair_r<float, gspn::kYSmem>(R, pl, dp, stream);
             } else {
-                err = launch_fused_r<__nv_bfloat16, false>(R, pl, dp, stream);
+                err = banded ? launch_pair_r<__nv_bfloat16, gspn::kYBanded>(R, pl, dp, stream)
+                             : launch_pair_r<__nv_bfloat16, gspn::kYSmem>(R, pl, dp, stream);
             }
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }

@@ -1,16 +1,17 @@
-// General Prop2D forward for shapes the fused kernel does not take (lines
-// longer than 256 positions, or bf16 rows of odd width, whose rows are not
-// 4-byte aligned).  Same work split as the fused kernel (a CTA of four
-// warps per plane band, warp d = direction d), but each warp keeps its
+// General Prop2D forward for shapes the paired kernel does not take (lines
+// longer than 256 positions, lines of one position, or bf16 rows of odd
+// width, whose rows are not 4-byte aligned).  A CTA of four warps owns a
+// plane band, warp d runs direction d; each warp keeps its
 // previous and current hidden line in shared memory, lanes stride over the
 // positions of a line, and inputs are read straight from global memory.
 // Correct for every size; not tuned.
 #pragma once
 
 #include "device_common.cuh"
-#include "prop2d_fused.cuh"
 
 namespace gspn {
+
+constexpr int kGenericThreads = 128;   // 4 warps: one per direction
 
 struct GenericParams {
     const void *x, *lam, *wl, *u;
@@ -22,7 +23,7 @@ struct GenericParams {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kFusedThreads)
+__global__ void __launch_bounds__(kGenericThreads)
 prop2d_generic_kernel(const GenericParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -41,7 +42,7 @@ prop2d_generic_kernel(const GenericParams p) {
     const T *WL = static_cast<const T *>(p.wl);
     const int Cw = p.share_w ? 1 : p.Cc;
 
-    for (int e = threadIdx.x; e < p.band_rows * YP; e += kFusedThreads) ys[e] = 0.0f;
+    for (int e = threadIdx.x; e < p.band_rows * YP; e += kGenericThreads) ys[e] = 0.0f;
     __syncthreads();
 
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
@@ -80,7 +81,7 @@ prop2d_generic_kernel(const GenericParams p) {
         T *outp = static_cast<T *>(p.out) + (static_cast<size_t>(b) * p.Cc + c) * HW +
                   static_cast<size_t>(band_lo) * W;
         const int n = (band_hi - band_lo) * W;
-        for (int e = threadIdx.x; e < n; e += kFusedThreads) {
+        for (int e = threadIdx.x; e < n; e += kGenericThreads) {
             const int i = e / W, j = e - i * W;
             outp[e] = from_f<T>(ys[i * YP + j]);
             ys[i * YP + j] = 0.0f;

@@ -173,11 +173,13 @@ def test_extreme_logits(gspn, mode, dtype):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "fused"),
-    ((1, 2, 256, 256), "f32", "fused-yglobal"),
-    ((1, 2, 256, 256), "bf16", "fused-banded"),
+    ((2, 3, 74, 74), "bf16", "pair"),
+    ((1, 2, 256, 256), "f32", "pair-yglobal"),
+    ((1, 2, 256, 256), "bf16", "pair-banded"),
     ((1, 2, 20, 33), "bf16", "generic"),       # odd bf16 row width
     ((1, 1, 300, 40), "f32", "generic"),       # line longer than 256
+    ((2, 2, 1, 40), "bf16", "generic"),        # lines of one position
+    ((1, 3, 17, 1), "f32", "generic"),
 ])
 def test_launch_paths(gspn, shape, dtype, path):
     B, Cc, H, W = shape
