@@ -95,8 +95,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity
 }
 
 __device__ __forceinline__ void red_add_shared_if(uint32_t addr, float v, bool pred) {
+    // No memory clobber: these only add into the output plane, which is read
+    // back after a barrier (itself ordered against every volatile asm here).
     asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p red.shared.add.f32 [%0], %1;\n}"
-                 ::"r"(addr), "f"(v), "r"(static_cast<uint32_t>(pred)) : "memory");
+                 ::"r"(addr), "f"(v), "r"(static_cast<uint32_t>(pred)));
 }
 
 // Copy the 4-byte words [w0, w0 + nwords) of a global buffer to shared

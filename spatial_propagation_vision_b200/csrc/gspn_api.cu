@@ -8,13 +8,13 @@
 #include <mutex>
 
 #include "gspn.h"
+#include "prop2d_dir.cuh"
 #include "prop2d_generic.cuh"
-#include "prop2d_pair.cuh"
 
 namespace {
 
+using gspn::DirParams;
 using gspn::GenericParams;
-using gspn::PairParams;
 
 struct LaunchInfo {
     int launches = 0, grid = 0, block = 0, smem = 0;
@@ -22,7 +22,7 @@ struct LaunchInfo {
 };
 thread_local LaunchInfo g_last;
 
-constexpr int kMaxPairLine = 256;       // longest line (H or W) the paired kernel holds in registers
+constexpr int kMaxDirLine = 256;        // longest line (H or W) the direction kernel holds in registers
 constexpr int kMaxGenericLine = 4096;   // longest line the general kernel accepts
 
 struct DeviceProps {
@@ -49,40 +49,39 @@ cudaError_t device_props(DeviceProps &dp) {
 
 inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
-// Launch geometry of the paired-direction kernel.
-struct PairPlan {
+// Launch geometry of the direction kernel.
+struct DirPlan {
     bool y_global = false;
     int smem = 0;
-    PairParams p{};
+    DirParams p{};
 };
 
-// Bytes of one (half, tensor) slot of the column ring (see ColLayout).
+// Bytes of one tensor slot of a column-ring stage (see ColLayout).
 int col_slot_bytes(int H, int R) {
     const int words = (R % 2) ? H * 4 : H * 5 + 32;
     return round_up(words * 4, 16);
 }
 
-// Choose the row chunk and the output mode so that one CTA fits `cap` bytes
-// of shared memory.  Output modes: the fp32 output plane in shared memory;
-// fp32 outputs accumulated in global memory (L2 atomics); row bands of the
-// output plane in shared memory (the scans are rerun per band).
-bool plan_pair_fit(PairPlan &pl, int cap, int H, int W, int dirs, int es, int R, bool allow_yg,
-                   int min_t_row) {
-    const bool row_on = dirs & 3, col_on = dirs & 12;
+// Choose the row chunk for output mode `mode` so that one CTA fits `cap`
+// bytes of shared memory.  Output modes: 0, the fp32 output plane in shared
+// memory; 1, fp32 outputs accumulated in global memory (L2 atomics); 2, row
+// bands of the output plane in shared memory (the scans are rerun per band).
+bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int es, int R, int only_mode,
+                  int min_t_row) {
+    const int n_row = ((dirs >> 0) & 1) + ((dirs >> 1) & 1);
+    const int n_col = ((dirs >> 2) & 1) + ((dirs >> 3) & 1);
     const int YP = W | 1;
     const int slot_col = col_slot_bytes(H, R);
-    const int col_ring = col_on ? gspn::kColStages * 2 * gspn::kPairTensors * slot_col : 0;
-    // mbarriers of the row ring and the shift table of its staged spans, then
-    // a tail that keeps reads of positions past the end of a line in bounds
-    // (256 bytes: 3 mbarriers at 0, shift table at 64, 12 source pointers at 128)
+    const int col_ring = gspn::kDirStages * gspn::kTensors * slot_col;
+    // mbarriers and span-shift tables (256 bytes), then a tail that keeps the
+    // reads of positions past the end of a line inside the allocation
     const int pad = 256 + round_up(32 * R * 20 + 64, 16);
-    for (int mode = 0; mode < 3; ++mode) {
-        if (mode == 1 && !allow_yg) continue;
+    for (int mode = only_mode; mode <= only_mode; ++mode) {
         for (int t_row = 8; t_row >= min_t_row; t_row >>= 1) {
             // a staged span starts at its source address modulo 16 and is rounded up to 16 bytes
             const int slot_row = round_up(t_row * W * es + 32, 16);
-            const int row_ring = row_on ? gspn::kRowStages * 2 * gspn::kPairTensors * slot_row : 0;
-            const int rings = row_ring + col_ring + pad;
+            const int row_ring = gspn::kDirStages * gspn::kTensors * slot_row;
+            const int rings = n_row * row_ring + n_col * col_ring + pad;
             int band_rows = H, y_bytes = 0;
             if (mode == 0) {
                 y_bytes = round_up(H * YP * 4, 16);
@@ -93,13 +92,17 @@ bool plan_pair_fit(PairPlan &pl, int cap, int H, int W, int dirs, int es, int R,
                 y_bytes = round_up(band_rows * YP * 4, 16);
             }
             if (y_bytes + rings > cap) continue;
-            PairParams &p = pl.p;
+            DirParams &p = pl.p;
             p.t_row = t_row;
             p.slot_row = slot_row;
             p.slot_col = slot_col;
-            p.ring_row = y_bytes;
-            p.ring_col = y_bytes + row_ring;
-            p.bar_off = y_bytes + row_ring + col_ring;
+            int off = y_bytes;
+            for (int d = 0; d < 4; ++d) {
+                if (!((dirs >> d) & 1)) { p.ring[d] = -1; continue; }
+                p.ring[d] = off;
+                off += d < 2 ? row_ring : col_ring;
+            }
+            p.bar_off = off;
             p.y_pitch = YP;
             p.band_rows = band_rows;
             p.bands = (H + band_rows - 1) / band_rows;
@@ -112,36 +115,36 @@ bool plan_pair_fit(PairPlan &pl, int cap, int H, int W, int dirs, int es, int R,
 }
 
 template <typename T, int R, int MODE>
-cudaError_t launch_pair_t(const PairPlan &pl, const DeviceProps &dp, cudaStream_t stream) {
-    auto kern = gspn::prop2d_pair_kernel<T, R, MODE>;
+cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t stream) {
+    auto kern = gspn::prop2d_dir_kernel<T, R, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kPairThreads, pl.smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kDirThreads, pl.smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = static_cast<long long>(dp.sms) * per_sm;
     if (grid > pl.p.n_items) grid = pl.p.n_items;
-    kern<<<static_cast<unsigned>(grid), gspn::kPairThreads, pl.smem, stream>>>(pl.p);
+    kern<<<static_cast<unsigned>(grid), gspn::kDirThreads, pl.smem, stream>>>(pl.p);
     g_last.launches = 1;
     g_last.grid = static_cast<int>(grid);
-    g_last.block = gspn::kPairThreads;
+    g_last.block = gspn::kDirThreads;
     g_last.smem = pl.smem;
-    g_last.path = MODE == gspn::kYGlobal ? "pair-yglobal" : MODE == gspn::kYBanded ? "pair-banded" : "pair";
+    g_last.path = MODE == gspn::kYGlobal ? "dir-yglobal" : MODE == gspn::kYBanded ? "dir-banded" : "dir";
     return cudaGetLastError();
 }
 
 template <typename T, int MODE>
-cudaError_t launch_pair_r(int R, const PairPlan &pl, const DeviceProps &dp, cudaStream_t s) {
+cudaError_t launch_dir_r(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s) {
     switch (R) {
-        case 1: return launch_pair_t<T, 1, MODE>(pl, dp, s);
-        case 2: return launch_pair_t<T, 2, MODE>(pl, dp, s);
-        case 3: return launch_pair_t<T, 3, MODE>(pl, dp, s);
-        case 4: return launch_pair_t<T, 4, MODE>(pl, dp, s);
-        case 5: return launch_pair_t<T, 5, MODE>(pl, dp, s);
-        case 6: return launch_pair_t<T, 6, MODE>(pl, dp, s);
-        case 7: return launch_pair_t<T, 7, MODE>(pl, dp, s);
-        case 8: return launch_pair_t<T, 8, MODE>(pl, dp, s);
+        case 1: return launch_dir_t<T, 1, MODE>(pl, dp, s);
+        case 2: return launch_dir_t<T, 2, MODE>(pl, dp, s);
+        case 3: return launch_dir_t<T, 3, MODE>(pl, dp, s);
+        case 4: return launch_dir_t<T, 4, MODE>(pl, dp, s);
+        case 5: return launch_dir_t<T, 5, MODE>(pl, dp, s);
+        case 6: return launch_dir_t<T, 6, MODE>(pl, dp, s);
+        case 7: return launch_dir_t<T, 7, MODE>(pl, dp, s);
+        case 8: return launch_dir_t<T, 8, MODE>(pl, dp, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -232,8 +235,7 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
     if (!x || !lambda || !wlogit || !u || !out) return GSPN_ERR_NULL;
     if (misaligned(x) || misaligned(lambda) || misaligned(wlogit) || misaligned(u) || misaligned(out))
         return GSPN_ERR_ALIGN;
-    // every element offset must fit the kernels' 64-bit indexing; planes and
-    // item counts must fit 32-bit ints
+    // planes, rows and item counts must fit 32-bit ints (element offsets are 64-bit)
     const long long HW = static_cast<long long>(H) * W;
     if (HW > (1LL << 30) || static_cast<long long>(B) * Cc * H > 0x7fffffffLL)
         return GSPN_ERR_SHAPE;
@@ -246,20 +248,27 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
 
     const int es = dtype == GSPN_BF16 ? 2 : 4;
     cudaError_t err = cudaSuccess;
-    const bool pair_ok = maxline <= kMaxPairLine && H >= 2 && W >= 2 && (es == 4 || (W % 2 == 0));
-    if (pair_ok) {
+    // bf16 rows of even width keep every row and span 4-byte aligned
+    const bool dir_ok = maxline <= kMaxDirLine && H >= 2 && W >= 2 && (es == 4 || (W % 2 == 0));
+    if (dir_ok) {
         const int R = (maxline + 31) / 32;
-        PairPlan pl;
+        DirPlan pl;
         pl.p.x = x; pl.p.lam = lambda; pl.p.wl = wlogit; pl.p.u = u; pl.p.out = out;
         pl.p.B = B; pl.p.Cc = Cc; pl.p.H = H; pl.p.W = W; pl.p.dirs = dirs; pl.p.share_w = share_w;
-        // Prefer three CTAs per SM, then two, then one; bands only as a last resort.
-        const int caps[3] = {dp.smem_per_sm / 3 - 1024, dp.smem_per_sm / 2 - 1024, dp.smem_optin};
+        // Output modes in order of preference (whole plane in shared memory,
+        // fp32 plane in global memory, bands: the last reruns the scans per
+        // band); within a mode, the most CTAs per SM that fit.
+        const int caps[4] = {dp.smem_per_sm / 4 - 1024, dp.smem_per_sm / 3 - 1024,
+                             dp.smem_per_sm / 2 - 1024, dp.smem_optin};
         bool fit = false;
-        for (int ci = 0; ci < 3 && !fit; ++ci) {
-            const int cap = caps[ci] < dp.smem_optin ? caps[ci] : dp.smem_optin;
-            fit = plan_pair_fit(pl, cap, H, W, dirs, es, R, es == 4, 2);
+        for (int mode = 0; mode < 3 && !fit; ++mode) {
+            if (mode == 1 && es != 4) continue;
+            for (int ci = 0; ci < 4 && !fit; ++ci) {
+                const int cap = caps[ci] < dp.smem_optin ? caps[ci] : dp.smem_optin;
+                fit = plan_dir_fit(pl, cap, H, W, dirs, es, R, mode, 2);
+            }
         }
-        if (!fit) fit = plan_pair_fit(pl, dp.smem_optin, H, W, dirs, es, R, es == 4, 1);
+        if (!fit) fit = plan_dir_fit(pl, dp.smem_optin, H, W, dirs, es, R, 2, 1);
         if (fit) {
             pl.p.n_items = B * Cc * pl.p.bands;
             const unsigned long long plane_bytes = static_cast<unsigned long long>(HW) * es;
@@ -268,12 +277,12 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
             pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane_bytes;
             const bool banded = pl.p.bands > 1;
             if (es == 4) {
-                err = pl.y_global ? launch_pair_r<float, gspn::kYGlobal>(R, pl, dp, stream)
-                      : banded    ? launch_pair_r<float, gspn::kYBanded>(R, pl, dp, stream)
-                                  : launch_pair_r<float, gspn::kYSmem>(R, pl, dp, stream);
+                err = pl.y_global ? launch_dir_r<float, gspn::kYGlobal>(R, pl, dp, stream)
+                      : banded    ? launch_dir_r<float, gspn::kYBanded>(R, pl, dp, stream)
+                                  : launch_dir_r<float, gspn::kYSmem>(R, pl, dp, stream);
             } else {
-                err = banded ? launch_pair_r<__nv_bfloat16, gspn::kYBanded>(R, pl, dp, stream)
-                             : launch_pair_r<__nv_bfloat16, gspn::kYSmem>(R, pl, dp, stream);
+                err = banded ? launch_dir_r<__nv_bfloat16, gspn::kYBanded>(R, pl, dp, stream)
+                             : launch_dir_r<__nv_bfloat16, gspn::kYSmem>(R, pl, dp, stream);
             }
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }

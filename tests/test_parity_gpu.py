@@ -173,9 +173,9 @@ def test_extreme_logits(gspn, mode, dtype):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "pair"),
-    ((1, 2, 256, 256), "f32", "pair-yglobal"),
-    ((1, 2, 256, 256), "bf16", "pair-banded"),
+    ((2, 3, 74, 74), "bf16", "dir"),
+    ((1, 2, 256, 256), "f32", "dir-yglobal"),
+    ((1, 2, 256, 256), "bf16", "dir-banded"),
     ((1, 2, 20, 33), "bf16", "generic"),       # odd bf16 row width
     ((1, 1, 300, 40), "f32", "generic"),       # line longer than 256
     ((2, 2, 1, 40), "bf16", "generic"),        # lines of one position
