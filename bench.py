@@ -44,6 +44,35 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_sources_sha() -> str:
+    """sha256 over the CUDA sources and the C-ABI header (sorted by name)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "spatial_propagation_vision_b200", "csrc", "*")) +
+                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was captured on the current kernel sources; else None."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"prop2d_dir_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    sha = re.search(r"kernel_sources_sha256:\s*([0-9a-f]{64})", text)
+    tb = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not sha or not tb or sha.group(1) != kernel_sources_sha():
+        return None
+    return int(tb.group(1))
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -336,10 +365,13 @@ def run_ours(args, w):
         "config": config_of(w, world),
         "hbm_frac_of_measured_peak": value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": args.traffic,
+                     "frac": achieved / peak,
+                     "traffic": args.traffic if args.traffic is not None else profiled_traffic(w.name),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch "
+                                       f"(profiles/prop2d_dir_{w.name}.md, same kernel sources) or null",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "prop2d_fused_kernel", "avg_launch_ms": avg_kernel_ms},
+                     "kernel": "prop2d_dir_kernel", "avg_launch_ms": avg_kernel_ms},
         "e2e": {"value": job_value(nbytes, world, e2e_ms * 1e-3), "unit": "GB/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "gspn_prop2d_fwd_host (pinned host buffers)"},
