@@ -73,24 +73,29 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uin
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
 }
+// Bulk prefetch of [src, src + bytes) into L2 (TMA engine); src 16-byte
+// aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Set by a kernel whose bounded wait for an asynchronous copy gave up (the
-// copy never completed); read and cleared by gspn_device_status().  The
-// library is one translation unit, so this is its only definition.
-__device__ unsigned int g_gspn_device_status = 0;
+// Bit set in the library's device status word (a __device__ variable of the
+// API translation unit whose address every launch passes in) by a kernel
+// whose bounded wait for an asynchronous copy gave up; read and cleared by
+// gspn_device_status().
 constexpr unsigned int kStatusCopyTimeout = 1u;
 constexpr long long kMaxWaitPolls = 1LL << 26;
 
 // Wait for phase `parity` of an mbarrier, polling at most kMaxWaitPolls
 // times; on timeout record it and return false (the caller carries on
 // with whatever the buffer holds, so the launch still terminates).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity, unsigned int *status) {
     for (long long i = 0; i < kMaxWaitPolls; ++i)
         if (mbar_try_wait(mbar, parity)) return true;
-    atomicOr(&g_gspn_device_status, kStatusCopyTimeout);
+    atomicOr(status, kStatusCopyTimeout);
     return false;
 }
 

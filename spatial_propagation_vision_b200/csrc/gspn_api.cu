@@ -8,26 +8,30 @@
 #include <mutex>
 
 #include "gspn.h"
-#include "prop2d_dir.cuh"
-#include "prop2d_generic.cuh"
+#include "launch.h"
 
 namespace {
 
 using gspn::DirParams;
 using gspn::GenericParams;
+using namespace gspn_host;
 
-struct LaunchInfo {
-    int launches = 0, grid = 0, block = 0, smem = 0;
-    const char *path = "none";
-};
 thread_local LaunchInfo g_last;
 
 constexpr int kMaxDirLine = 256;        // longest line (H or W) the direction kernel holds in registers
 constexpr int kMaxGenericLine = 4096;   // longest line the general kernel accepts
 
-struct DeviceProps {
-    int sms = 0, smem_optin = 0, smem_per_sm = 0, major = 0, minor = 0;
-};
+}  // namespace
+
+// Device status word of the library: bit kStatusCopyTimeout is set by a
+// kernel whose bounded wait for an asynchronous copy gave up.
+__device__ unsigned int g_gspn_device_status = 0;
+
+namespace {
+
+cudaError_t status_word(unsigned int **ptr) {
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(ptr), g_gspn_device_status);
+}
 
 cudaError_t device_props(DeviceProps &dp) {
     int dev = 0;
@@ -47,141 +51,44 @@ cudaError_t device_props(DeviceProps &dp) {
     return cudaSuccess;
 }
 
-inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
-
-// Launch geometry of the direction kernel.
-struct DirPlan {
-    bool y_global = false;
-    int smem = 0;
-    DirParams p{};
-};
-
-// Bytes of one tensor slot of a column-ring stage (see ColLayout).
-int col_slot_bytes(int H, int R) {
-    const int words = (R % 2) ? H * 4 : H * 5 + 32;
-    return round_up(words * 4, 16);
-}
-
-// Choose the row chunk for output mode `mode` so that one CTA fits `cap`
-// bytes of shared memory.  Output modes: 0, the fp32 output plane in shared
-// memory; 1, fp32 outputs accumulated in global memory (L2 atomics); 2, row
-// bands of the output plane in shared memory (the scans are rerun per band).
-bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int es, int R, int only_mode,
-                  int min_t_row) {
-    const int n_row = ((dirs >> 0) & 1) + ((dirs >> 1) & 1);
+// Shared-memory plan for output mode `mode` so that one CTA fits `cap`
+// bytes.  Output modes: 0, the fp32 output plane in shared memory; 1, fp32
+// outputs accumulated in global memory (L2 atomics); 2, row bands of the
+// output plane in shared memory (the scans are rerun per band).  Layout:
+// output plane or band, the column rings of the enabled column directions,
+// then the column warps' plane-pointer tables.
+bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
     const int n_col = ((dirs >> 2) & 1) + ((dirs >> 3) & 1);
-    const int YP = W | 1;
-    const int slot_col = col_slot_bytes(H, R);
-    const int col_ring = gspn::kDirStages * gspn::kTensors * slot_col;
-    // mbarriers and span-shift tables (256 bytes), then a tail that keeps the
-    // reads of positions past the end of a line inside the allocation
-    const int pad = 256 + round_up(32 * R * 20 + 64, 16);
-    for (int mode = only_mode; mode <= only_mode; ++mode) {
-        for (int t_row = 8; t_row >= min_t_row; t_row >>= 1) {
-            // a staged span starts at its source address modulo 16 and is rounded up to 16 bytes
-            const int slot_row = round_up(t_row * W * es + 32, 16);
-            const int row_ring = gspn::kDirStages * gspn::kTensors * slot_row;
-            const int rings = n_row * row_ring + n_col * col_ring + pad;
-            int band_rows = H, y_bytes = 0;
-            if (mode == 0) {
-                y_bytes = round_up(H * YP * 4, 16);
-            } else if (mode == 2) {
-                if (cap - rings < YP * 4) continue;
-                band_rows = (cap - rings) / (YP * 4);
-                if (band_rows > H) band_rows = H;
-                y_bytes = round_up(band_rows * YP * 4, 16);
-            }
-            if (y_bytes + rings > cap) continue;
-            DirParams &p = pl.p;
-            p.t_row = t_row;
-            p.slot_row = slot_row;
-            p.slot_col = slot_col;
-            int off = y_bytes;
-            for (int d = 0; d < 4; ++d) {
-                if (!((dirs >> d) & 1)) { p.ring[d] = -1; continue; }
-                p.ring[d] = off;
-                off += d < 2 ? row_ring : col_ring;
-            }
-            p.bar_off = off;
-            p.y_pitch = YP;
-            p.band_rows = band_rows;
-            p.bands = (H + band_rows - 1) / band_rows;
-            pl.smem = y_bytes + rings;
-            pl.y_global = mode == 1;
-            return true;
-        }
+    // odd pitch above every swizzled column index (see ycol)
+    const int YP = (W % 2 == 0) ? W + 1 : W + 2;
+    const int stage_col = round_up(H * gspn::kColPitch, 16);
+    const int col_ring = gspn::kColStages * stage_col;
+    const int rings = n_col * col_ring + gspn::kDirBarBytes;
+    int band_rows = H, y_bytes = 0;
+    if (mode == 0) {
+        y_bytes = round_up(H * YP * 4, 16);
+    } else if (mode == 2) {
+        if (cap - rings < YP * 4) return false;
+        band_rows = (cap - rings) / (YP * 4);
+        if (band_rows > H) band_rows = H;
+        y_bytes = round_up(band_rows * YP * 4, 16);
     }
-    return false;
-}
-
-template <typename T, int R, int MODE>
-cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t stream) {
-    auto kern = gspn::prop2d_dir_kernel<T, R, MODE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kDirThreads, pl.smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    long long grid = static_cast<long long>(dp.sms) * per_sm;
-    if (grid > pl.p.n_items) grid = pl.p.n_items;
-    kern<<<static_cast<unsigned>(grid), gspn::kDirThreads, pl.smem, stream>>>(pl.p);
-    g_last.launches = 1;
-    g_last.grid = static_cast<int>(grid);
-    g_last.block = gspn::kDirThreads;
-    g_last.smem = pl.smem;
-    g_last.path = MODE == gspn::kYGlobal ? "dir-yglobal" : MODE == gspn::kYBanded ? "dir-banded" : "dir";
-    return cudaGetLastError();
-}
-
-template <typename T, int MODE>
-cudaError_t launch_dir_r(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s) {
-    switch (R) {
-        case 1: return launch_dir_t<T, 1, MODE>(pl, dp, s);
-        case 2: return launch_dir_t<T, 2, MODE>(pl, dp, s);
-        case 3: return launch_dir_t<T, 3, MODE>(pl, dp, s);
-        case 4: return launch_dir_t<T, 4, MODE>(pl, dp, s);
-        case 5: return launch_dir_t<T, 5, MODE>(pl, dp, s);
-        case 6: return launch_dir_t<T, 6, MODE>(pl, dp, s);
-        case 7: return launch_dir_t<T, 7, MODE>(pl, dp, s);
-        case 8: return launch_dir_t<T, 8, MODE>(pl, dp, s);
-        default: return cudaErrorInvalidValue;
+    if (y_bytes + rings > cap) return false;
+    DirParams &p = pl.p;
+    p.stage_col = stage_col;
+    int off = y_bytes;
+    for (int d = 0; d < 4; ++d) {
+        if (d < 2 || !((dirs >> d) & 1)) { p.ring[d] = -1; continue; }
+        p.ring[d] = off;
+        off += col_ring;
     }
-}
-
-template <typename T>
-cudaError_t launch_generic(const GenericParams &gp0, const DeviceProps &dp, cudaStream_t stream,
-                           bool &fits) {
-    GenericParams gp = gp0;
-    const int YP = gp.W | 1;
-    gp.y_pitch = YP;
-    gp.hline = round_up(gp.H > gp.W ? gp.H : gp.W, 4);
-    const int hbytes = 4 * 2 * gp.hline * 4;
-    const int cap = dp.smem_optin;
-    int band_rows = (cap - hbytes) / (YP * 4);
-    fits = band_rows >= 1;
-    if (!fits) return cudaSuccess;
-    if (band_rows > gp.H) band_rows = gp.H;
-    gp.band_rows = band_rows;
-    gp.bands = (gp.H + band_rows - 1) / band_rows;
-    gp.n_items = gp.B * gp.Cc * gp.bands;
-    const int smem = round_up(band_rows * YP * 4, 16) + hbytes;
-    auto kern = gspn::prop2d_generic_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kGenericThreads, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    long long grid = static_cast<long long>(dp.sms) * per_sm;
-    if (grid > gp.n_items) grid = gp.n_items;
-    kern<<<static_cast<unsigned>(grid), gspn::kGenericThreads, smem, stream>>>(gp);
-    g_last.launches = 1;
-    g_last.grid = static_cast<int>(grid);
-    g_last.block = gspn::kGenericThreads;
-    g_last.smem = smem;
-    g_last.path = "generic";
-    return cudaGetLastError();
+    p.bar_off = off;
+    p.y_pitch = YP;
+    p.band_rows = band_rows;
+    p.bands = (H + band_rows - 1) / band_rows;
+    pl.smem = y_bytes + rings;
+    pl.y_global = mode == 1;
+    return true;
 }
 
 bool misaligned(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) != 0; }
@@ -190,11 +97,11 @@ bool misaligned(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15
 
 extern "C" gspn_status gspn_device_status(unsigned int *flags, int clear) {
     if (!flags) return GSPN_ERR_NULL;
-    if (cudaMemcpyFromSymbol(flags, gspn::g_gspn_device_status, sizeof(unsigned int)) != cudaSuccess)
+    if (cudaMemcpyFromSymbol(flags, g_gspn_device_status, sizeof(unsigned int)) != cudaSuccess)
         return GSPN_ERR_CUDA;
     if (clear) {
         const unsigned int zero = 0;
-        if (cudaMemcpyToSymbol(gspn::g_gspn_device_status, &zero, sizeof(unsigned int)) != cudaSuccess)
+        if (cudaMemcpyToSymbol(g_gspn_device_status, &zero, sizeof(unsigned int)) != cudaSuccess)
             return GSPN_ERR_CUDA;
     }
     return GSPN_OK;
@@ -265,24 +172,24 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
             if (mode == 1 && es != 4) continue;
             for (int ci = 0; ci < 4 && !fit; ++ci) {
                 const int cap = caps[ci] < dp.smem_optin ? caps[ci] : dp.smem_optin;
-                fit = plan_dir_fit(pl, cap, H, W, dirs, es, R, mode, 2);
+                fit = plan_dir_fit(pl, cap, H, W, dirs, mode);
             }
         }
-        if (!fit) fit = plan_dir_fit(pl, dp.smem_optin, H, W, dirs, es, R, 2, 1);
         if (fit) {
             pl.p.n_items = B * Cc * pl.p.bands;
             const unsigned long long plane_bytes = static_cast<unsigned long long>(HW) * es;
             pl.p.end_x = static_cast<unsigned long long>(B) * Cc * plane_bytes;
             pl.p.end_gate = 4ULL * pl.p.end_x;
             pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane_bytes;
+            if (status_word(&pl.p.status) != cudaSuccess) return GSPN_ERR_CUDA;
             const bool banded = pl.p.bands > 1;
             if (es == 4) {
-                err = pl.y_global ? launch_dir_r<float, gspn::kYGlobal>(R, pl, dp, stream)
-                      : banded    ? launch_dir_r<float, gspn::kYBanded>(R, pl, dp, stream)
-                                  : launch_dir_r<float, gspn::kYSmem>(R, pl, dp, stream);
+                err = pl.y_global ? launch_dir_f32_global(R, pl, dp, stream, g_last)
+                      : banded    ? launch_dir_f32_banded(R, pl, dp, stream, g_last)
+                                  : launch_dir_f32_smem(R, pl, dp, stream, g_last);
             } else {
-                err = banded ? launch_dir_r<__nv_bfloat16, gspn::kYBanded>(R, pl, dp, stream)
-                             : launch_dir_r<__nv_bfloat16, gspn::kYSmem>(R, pl, dp, stream);
+                err = banded ? launch_dir_bf16_banded(R, pl, dp, stream, g_last)
+                             : launch_dir_bf16_smem(R, pl, dp, stream, g_last);
             }
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }
@@ -291,8 +198,7 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
     gp.x = x; gp.lam = lambda; gp.wl = wlogit; gp.u = u; gp.out = out;
     gp.B = B; gp.Cc = Cc; gp.H = H; gp.W = W; gp.dirs = dirs; gp.share_w = share_w;
     bool fits = false;
-    err = es == 4 ? launch_generic<float>(gp, dp, stream, fits)
-                  : launch_generic<__nv_bfloat16>(gp, dp, stream, fits);
+    err = launch_generic(gp, es == 2, dp, stream, fits, g_last);
     if (!fits) return GSPN_ERR_SHAPE;
     return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
 }

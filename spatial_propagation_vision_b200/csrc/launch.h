@@ -1,0 +1,46 @@
+// Host-side plumbing shared by the library's translation units: launch
+// geometry, device properties and the per-variant launch functions.  Each
+// (element type, output mode) variant of the direction kernel is compiled
+// in its own translation unit so the library builds in parallel.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "prop2d_dir.cuh"
+#include "prop2d_generic.cuh"
+
+namespace gspn_host {
+
+// What the last gspn_prop2d_fwd call on this host thread launched.
+struct LaunchInfo {
+    int launches = 0, grid = 0, block = 0, smem = 0;
+    const char *path = "none";
+};
+
+struct DeviceProps {
+    int sms = 0, smem_optin = 0, smem_per_sm = 0, major = 0, minor = 0;
+};
+
+// Launch geometry of the direction kernel.
+struct DirPlan {
+    bool y_global = false;
+    int smem = 0;
+    gspn::DirParams p{};
+};
+
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// Direction kernel, one function per (element type, output mode); R is the
+// positions per lane (1..8).
+cudaError_t launch_dir_f32_smem(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_f32_banded(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_f32_global(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_smem(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_banded(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+
+// General kernel; `fits` is false when even one output row does not fit.
+cudaError_t launch_generic(const gspn::GenericParams &gp, bool bf16, const DeviceProps &dp,
+                           cudaStream_t stream, bool &fits, LaunchInfo &li);
+
+}  // namespace gspn_host

@@ -5,10 +5,9 @@
 // warp d runs direction d: 0 top->bottom, 1 bottom->top (row lines),
 // 2 left->right, 3 right->left (column lines).  Lane l holds the R
 // consecutive positions q = l*R + r of the current line in registers; the
-// neighbours across lanes come from shuffles.  Four independent warps per
-// plane give the scheduler enough warps to hide the latency of the
-// dependent arithmetic (the kernel is bound by instruction issue, not by
-// memory), and pairs of positions share packed f32x2 instructions.
+// neighbours across lanes come from shuffles.  Each warp runs code compiled
+// for its own direction (orientation and sweep sign are template
+// parameters), so the line and offset arithmetic inside a chunk is static.
 //
 // Normalisation (Sec. 5.1 "Fused CUDA normalization": sigmoid, local sum,
 // clamp, divide), folded into the update.  With a_k = 1 + exp(-z_k),
@@ -18,25 +17,39 @@
 // which takes three exponentials and one reciprocal per position.  An
 // off-grid slot takes a_k = 1, P_k = 0.  Whenever the clamp of the
 // denominator could bind, or a product overflows, D exceeds a threshold
-// (1e11 with three on-grid slots, 1e5 with two) or is not finite, and the
-// line is recomputed in the plain form.  The weights of line s+1 do not
-// depend on the hidden line; they are computed in the same straight block
-// as line s's recurrence so the two chains interleave.
+// (1e11 with three on-grid slots, 1e5 with two) or is not finite; the
+// weights of that line are then recomputed in the plain form.  The weights
+// of line s+1 do not depend on the hidden state; they are computed in the
+// same straight block as line s's update, and the weight sets of
+// consecutive lines alternate between two register sets.
 //
-// Input lines are staged in shared memory, several lines per chunk, in a
-// two-stage ring per warp:
-//   * row lines: the rows of a chunk are one contiguous span per tensor;
-//     lane t < 6 moves tensor t's span with one bulk copy (TMA engine) into a
-//     16-byte aligned slot and arrives on the stage's mbarrier;
-//   * column lines: a strip of 16 bytes of every row (8 bf16 / 4 fp32
-//     columns) moved by the lanes with 4-byte cp.async; a strip row takes 4
-//     words, XOR-swizzled by row so that the lanes reading one column hit
-//     distinct banks (odd R), or 5 words plus one word per lane (even R).
+// Input staging in shared memory:
+//   * row lines: a chunk of t_row rows is one contiguous span per tensor;
+//     lane t < 6 moves tensor t's span with one bulk copy (TMA engine) into
+//     a 16-byte aligned slot of a three-stage ring and arrives on the
+//     stage's mbarrier; the lanes then read their positions of a line with
+//     16-bit loads;
+//   * column lines: a chunk is a strip of 16 bytes of every grid row (8 bf16
+//     or 4 fp32 columns).  The strip rows of the six tensors are interleaved
+//     (104-byte pitch: six 16-byte pieces and 8 bytes of padding, so that
+//     the lanes' 8-byte reads hit distinct banks).  Each lane copies
+//     (4-byte cp.async) and later reads its own R rows, so it waits for its
+//     own copies only.  One 8-byte read per tensor and position brings half
+//     a strip (4 bf16 / 2 fp32 columns) into registers.  Right-to-left
+//     scans store the words of a strip row in reverse order, so both sweeps
+//     meet their columns in scan order.
 // The gated outputs u * h of the four directions are summed into one fp32
 // plane in shared memory with shared-memory atomics and written once.
+//
+// Positions past the end of a line (q >= M) compute finite garbage that
+// never reaches a valid position: their right-hand neighbour term of
+// position M-1 has P_2 = 0.  For that they read finite values only: the
+// rings are zeroed at launch and afterwards hold copies of the inputs
+// (column lanes past the end read grid row 0's strip).
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
@@ -44,9 +57,11 @@
 namespace gspn {
 
 constexpr int kDirThreads = 128;   // warp d runs direction d
-constexpr int kDirStages = 2;      // ring depth per warp
-constexpr int kColWords = 4;       // 16 bytes of each row per column chunk
+constexpr int kColStages = 2;      // column ring depth
 constexpr int kTensors = 6;        // lambda, u, logit0, logit1, logit2, x
+constexpr int kColStrip = 16;      // bytes of each grid row per column chunk
+constexpr int kColPitch = 104;     // bytes per grid row of a column stage: 6 x 16 + 8
+constexpr int kDirBarBytes = 256;  // plane-pointer tables of the column warps
 
 // Output modes.
 constexpr int kYSmem = 0;     // whole fp32 output plane in shared memory
@@ -58,23 +73,12 @@ struct DirParams {
     void *out;
     int B, Cc, H, W, dirs, share_w;
     int n_items, bands, band_rows;
-    int t_row;                  // rows per row-line chunk
-    int slot_row, slot_col;     // bytes per tensor slot of a row / column ring stage
-    int ring[4];                // byte offset of direction d's ring (-1: direction off)
-    int bar_off;                // byte offset of the mbarriers and shift tables (256 bytes)
-    int y_pitch;                // floats per staged output row (odd)
+    int stage_col;              // bytes per column ring stage
+    int ring[4];                // byte offset of column direction d's ring (-1: none)
+    int bar_off;                // byte offset of the column warps' plane-pointer tables
+    int y_pitch;                // floats per staged output row (odd, > every ycol(j), j < W)
     unsigned long long end_x, end_gate, end_wl;   // byte sizes of x, lambda/u, logits
-};
-
-// Column-strip geometry: word address (relative to its slot) of word w of
-// strip row q.
-template <int R>
-struct ColLayout {
-    static constexpr bool kSwizzle = (R % 2) == 1;
-    static __device__ __forceinline__ int word(int q, int w) {
-        if (kSwizzle) return q * 4 + (w ^ ((q / (8 * R)) & 3));
-        return q * 5 + q / R + w;
-    }
+    unsigned int *status;       // device status word (bounded waits that gave up)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -118,334 +122,667 @@ __device__ __forceinline__ unsigned long long dir_tensor_bytes(const DirParams &
 template <int R>
 struct LineW {
     float P0[R], P1[R], P2[R], rD[R], bx[R], uu[R];
-    bool bad;   // some position needs the plain form
 };
 
-template <typename T, int R, bool ROW, int MODE>
-struct DirWarp {
-    static constexpr int es = sizeof(T);
-    static constexpr int NS = kDirStages;
-    static constexpr int kColRows = (32 * R + 32 / kColWords - 1) / (32 / kColWords);  // strip rows per lane
-
-    const DirParams &p;
-    const int lane;
-    const int D;                    // direction slot (0..3)
-    const bool fwd;                 // sweeps forward (top->bottom / left->right)
-    unsigned char *const ring;
-    const uint32_t bars;            // this warp's NS mbarriers (row lines)
-    unsigned char *const shifts;    // this warp's [stage][tensor] span shifts (row lines)
-    const int slot;
-    const int L, M, T_, nch;
-    // source planes of the item whose chunks are being issued
-    int issue_item;
-    const char *my_gp;              // row lines: lane t < 6 keeps tensor t's plane
-    const char *gtab[kTensors];     // column lines: every lane copies every tensor
-    int col_off[kColRows];          // strip-row word offsets of this lane's rows (column lines)
-
-    __device__ DirWarp(const DirParams &p_, unsigned char *smem_, int lane_, int d_)
-        : p(p_), lane(lane_), D(d_), fwd((d_ % 2) == 0),
-          ring(smem_ + (d_ == 0 ? p_.ring[0] : d_ == 1 ? p_.ring[1] : d_ == 2 ? p_.ring[2] : p_.ring[3])),
-          bars(smem_u32(smem_ + p_.bar_off) + 8 * NS * D),
-          shifts(smem_ + p_.bar_off + 64 + 16 * D),
-          slot(ROW ? p_.slot_row : p_.slot_col),
-          L(ROW ? p_.H : p_.W), M(ROW ? p_.W : p_.H),
-          T_(ROW ? p_.t_row : kColWords * 4 / es),
-          nch(((ROW ? p_.H : p_.W) + (ROW ? p_.t_row : kColWords * 4 / es) - 1) /
-              (ROW ? p_.t_row : kColWords * 4 / es)),
-          issue_item(-1), my_gp(nullptr) {
-        if (!ROW) {
-            const int w = lane & (kColWords - 1), i0 = lane / kColWords;
-#pragma unroll
-            for (int k = 0; k < kColRows; ++k) col_off[k] = 4 * ColLayout<R>::word(i0 + k * (32 / kColWords), w);
-        }
-    }
-
-    // Lines [lo, hi) of chunk c in grid coordinates.
-    __device__ __forceinline__ void chunk(int c, int &lo, int &hi) const {
-        if (fwd) {
-            lo = c * T_;
-            hi = min(L, lo + T_);
-        } else {
-            hi = L - c * T_;
-            lo = max(0, hi - T_);
-        }
-    }
-
-    __device__ __forceinline__ unsigned char *slot_ptr(int stage, int t) const {
-        return ring + (stage * kTensors + t) * slot;
-    }
-
-    __device__ __forceinline__ void set_issue_item(int item) {
-        if (item == issue_item) return;
-        issue_item = item;
-        const int plane = item / p.bands;
-        const int b = plane / p.Cc, ch = plane - b * p.Cc;
-        if (ROW) {
-            if (lane < kTensors) my_gp = dir_tensor(p, lane) + dir_plane(p, b, ch, D, lane) * es;
-        } else {
-#pragma unroll
-            for (int t = 0; t < kTensors; ++t) gtab[t] = dir_tensor(p, t) + dir_plane(p, b, ch, D, t) * es;
-        }
-    }
-
-    // Issue the copies of chunk c of `item` into ring stage `stage`.  Every
-    // read of that stage has completed: its values were consumed by
-    // instructions issued before this point.
-    __device__ __forceinline__ void issue(int item, int c, int stage) {
-        set_issue_item(item);
-        int lo, hi;
-        chunk(c, lo, hi);
-        if (ROW) {
-            if (lane < kTensors) {
-                const int t = lane;
-                const char *s = my_gp + static_cast<size_t>(lo) * p.W * es;
-                const uint32_t sh = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(s) & 15);
-                const char *a = s - sh;
-                uint32_t n = (sh + static_cast<uint32_t>((hi - lo) * p.W * es) + 15u) & ~15u;
-                int tl = 0;
-                // never read past the end of the tensor: the last partial 16 bytes
-                // are then copied by hand
-                const unsigned long long end = dir_tensor_bytes(p, t);
-                const unsigned long long off = static_cast<unsigned long long>(a - dir_tensor(p, t));
-                if (off + n > end) {
-                    tl = static_cast<int>(end - (off + n - 16));
-                    n -= 16;
-                }
-                unsigned char *dst = slot_ptr(stage, t);
-                shifts[stage * 8 + t] = static_cast<unsigned char>(sh);
-                for (int e = 0; e < tl; e += 2)   // rare: end of the tensor
-                    *reinterpret_cast<unsigned short *>(dst + n + e) =
-                        *reinterpret_cast<const unsigned short *>(a + n + e);
-                const uint32_t bar = bars + 8 * stage;
-                mbar_arrive_expect_tx(bar, n);
-                if (n) bulk_copy_g2s(smem_u32(dst), a, n, bar);
-            }
-        } else {
-            const int w = lane & (kColWords - 1), i0 = lane / kColWords;
-            const int nw = ((hi - lo) * es) >> 2;   // words per row segment, <= kColWords
-            if (w < nw) {
-                const size_t gstep = static_cast<size_t>(32 / kColWords) * p.W * es;
-                const size_t lane_off = (static_cast<size_t>(i0) * p.W + lo) * es + 4 * w;
-#pragma unroll
-                for (int t = 0; t < kTensors; ++t) {
-                    const char *s = gtab[t] + lane_off;
-                    const uint32_t sb = smem_u32(slot_ptr(stage, t));
-#pragma unroll
-                    for (int k = 0; k < kColRows; ++k) {
-                        if (i0 + k * (32 / kColWords) < p.H) cp_async_4(sb + col_off[k], s);
-                        s += gstep;
-                    }
-                }
-            }
-            cp_async_commit();
-        }
-    }
-
-    // Wait until the g-th chunk of this warp (in `stage`) has landed.
-    __device__ __forceinline__ void wait_chunk(int g, int stage) const {
-        if (ROW) {
-            mbar_wait_bounded(bars + 8 * stage, static_cast<uint32_t>((g / NS) & 1));
-        } else {
-            cp_async_wait<NS - 2>();
-            __syncwarp();
-        }
-    }
-
-    // Shared-memory address of line li's element at position lane*R + r.
-    __device__ __forceinline__ const unsigned char *elem(const unsigned char *slotp, int shift,
-                                                         int li, int r) const {
-        if (ROW) return slotp + shift + (li * p.W + lane * R + r) * es;
-        const int q = lane * R + r;
-        return slotp + 4 * ColLayout<R>::word(q, (li * es) >> 2) + ((li * es) & 3);
-    }
-
-    // Raw inputs of line li of the current chunk -> normalisation terms.
-    __device__ __forceinline__ void weights(const unsigned char *const (&sp)[kTensors],
-                                            const int (&shift)[kTensors], int li,
-                                            const float (&m0)[R], const float (&m2)[R],
-                                            const float (&ithr)[R], const bool (&valid)[R],
-                                            LineW<R> &W) const {
-        float v[kTensors][R];
-#pragma unroll
-        for (int t = 0; t < kTensors; ++t)
-#pragma unroll
-            for (int r = 0; r < R; ++r) v[t][r] = sload<T>(elem(sp[t], shift[t], li, r));
-        constexpr float nl2e = -1.4426950408889634f;
-        bool bad = false;
-        // positions (r, r+1) as one f32x2 pair; a last odd position alone
-#pragma unroll
-        for (int r = 0; r + 1 < R; r += 2) {
-            const float2 n2 = make_float2(nl2e, nl2e);
-            const float2 one2 = make_float2(1.0f, 1.0f);
-            const float2 t0 = __fmul2_rn(make_float2(v[2][r], v[2][r + 1]), n2);
-            const float2 t1 = __fmul2_rn(make_float2(v[3][r], v[3][r + 1]), n2);
-            const float2 t2 = __fmul2_rn(make_float2(v[4][r], v[4][r + 1]), n2);
-            const float2 a0 = __ffma2_rn(make_float2(ex2(t0.x), ex2(t0.y)), make_float2(m0[r], m0[r + 1]), one2);
-            const float2 a1 = __fadd2_rn(make_float2(ex2(t1.x), ex2(t1.y)), one2);
-            const float2 a2 = __ffma2_rn(make_float2(ex2(t2.x), ex2(t2.y)), make_float2(m2[r], m2[r + 1]), one2);
-            const float2 P0 = __fmul2_rn(__fmul2_rn(a1, a2), make_float2(m0[r], m0[r + 1]));
-            const float2 P1 = __fmul2_rn(a0, a2);
-            const float2 P2 = __fmul2_rn(__fmul2_rn(a0, a1), make_float2(m2[r], m2[r + 1]));
-            const float2 Dn = __fadd2_rn(__fadd2_rn(P0, P1), P2);
-            const float2 k = __fmul2_rn(Dn, make_float2(ithr[r], ithr[r + 1]));
-            // over the threshold, or NaN (an off-grid slot whose exponential overflowed)
-            bad = bad || (valid[r] && !(k.x <= 1.0f)) || (valid[r + 1] && !(k.y <= 1.0f));
-            const float2 bx = __fmul2_rn(make_float2(v[0][r], v[0][r + 1]), make_float2(v[5][r], v[5][r + 1]));
-            W.P0[r] = P0.x; W.P0[r + 1] = P0.y;
-            W.P1[r] = P1.x; W.P1[r + 1] = P1.y;
-            W.P2[r] = P2.x; W.P2[r + 1] = P2.y;
-            W.rD[r] = rcp(Dn.x); W.rD[r + 1] = rcp(Dn.y);
-            W.bx[r] = bx.x; W.bx[r + 1] = bx.y;
-            W.uu[r] = v[1][r]; W.uu[r + 1] = v[1][r + 1];
-        }
-        if (R % 2) {
-            const int r = R - 1;
-            const float a0 = fmaf(ex2(v[2][r] * nl2e), m0[r], 1.0f);
-            const float a1 = ex2(v[3][r] * nl2e) + 1.0f;
-            const float a2 = fmaf(ex2(v[4][r] * nl2e), m2[r], 1.0f);
-            const float P0 = a1 * a2 * m0[r];
-            const float P1 = a0 * a2;
-            const float P2 = a0 * a1 * m2[r];
-            const float Dn = (P0 + P1) + P2;
-            bad = bad || (valid[r] && !(Dn * ithr[r] <= 1.0f));
-            W.P0[r] = P0;
-            W.P1[r] = P1;
-            W.P2[r] = P2;
-            W.rD[r] = rcp(Dn);
-            W.bx[r] = v[0][r] * v[5][r];
-            W.uu[r] = v[1][r];
-        }
-        W.bad = bad;
-    }
-
-    // Plain-form update of line li for every position (rare path).
-    __device__ __forceinline__ void plain_line(const unsigned char *const (&sp)[kTensors],
-                                               const int (&shift)[kTensors], int li,
-                                               const float (&h)[R], float hl, float hr,
-                                               float (&hn)[R]) const {
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int q = lane * R + r;
-            const float left = r > 0 ? h[r - 1] : hl;
-            const float right = r < R - 1 ? h[r + 1] : hr;
-            float v[kTensors];
-#pragma unroll
-            for (int t = 0; t < kTensors; ++t) v[t] = sload<T>(elem(sp[t], shift[t], li, r));
-            const W3 w = normalise_plain(v[2], v[3], v[4], q > 0, q + 1 < M);
-            float acc = v[0] * v[5];
-            if (q > 0) acc = fmaf(w.w0, left, acc);
-            acc = fmaf(w.w1, h[r], acc);
-            if (q + 1 < M) acc = fmaf(w.w2, right, acc);
-            hn[r] = acc;
-        }
-    }
-
-    // Run every line of `item`.  `g` counts this warp's chunks in the launch
-    // (ring position); `total` is the number of chunks it runs in the launch.
-    __device__ void run_item(int item, int &g, int total, float *ys, float *yg, int band_lo,
-                             int band_hi) {
-        float m0[R], m2[R], ithr[R];
-        bool valid[R], inband[R];
+// Per-lane constants of a line of M positions.
+template <int R>
+struct LaneGeom {
+    float m0[R], m2[R];   // 1 where the slot k = 0 / k = 2 neighbour is on the grid
+    int thr[R];           // bit pattern of the fast-form threshold on D
+    bool valid[R];        // q < M
+    __device__ __forceinline__ void init(int lane, int M) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int q = lane * R + r;
             valid[r] = q < M;
             m0[r] = q > 0 ? 1.0f : 0.0f;
             m2[r] = q + 1 < M ? 1.0f : 0.0f;
-            ithr[r] = (q > 0 && q + 1 < M) ? 1e-11f : 1e-5f;
-            inband[r] = valid[r] && (ROW || MODE != kYBanded || (q >= band_lo && q < band_hi));
+            thr[r] = __float_as_int((q > 0 && q + 1 < M) ? 1e11f : 1e5f);
         }
-        const uint32_t ysa = smem_u32(ys);
-        float hs[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) hs[r] = 0.0f;
+    }
+};
 
-        const unsigned char *sp[kTensors];
-        int shift[kTensors];
-        int lo = 0, nl = 0;
-        auto enter_chunk = [&](int c) {
-            const int stage = g % NS;
-            wait_chunk(g, stage);
-            if (g + NS - 1 < total) {
-                const int gn = g + NS - 1;
-                const int kk = gn / nch;
-                issue(blockIdx.x + kk * gridDim.x, gn - kk * nch, gn % NS);
-            } else if (!ROW) {
-                cp_async_commit();
+// Raw inputs of one line -> normalisation terms.  Returns true when some
+// position is outside the fast form's range: D above its threshold, or not
+// finite (as bit patterns, +inf and the hardware's NaN compare above every
+// threshold).  Positions past the end of the line take part; a flagged line
+// is simply recomputed in the plain form.
+template <int R>
+__device__ __forceinline__ bool line_weights(const float (&v)[kTensors][R], const LaneGeom<R> &g,
+                                             LineW<R> &W) {
+    constexpr float nl2e = -1.4426950408889634f;
+    bool bad = false;
+#pragma unroll
+    for (int r = 0; r + 1 < R; r += 2) {
+        const float2 n2 = make_float2(nl2e, nl2e);
+        const float2 one2 = make_float2(1.0f, 1.0f);
+        const float2 mm0 = make_float2(g.m0[r], g.m0[r + 1]);
+        const float2 mm2 = make_float2(g.m2[r], g.m2[r + 1]);
+        const float2 t0 = __fmul2_rn(make_float2(v[2][r], v[2][r + 1]), n2);
+        const float2 t1 = __fmul2_rn(make_float2(v[3][r], v[3][r + 1]), n2);
+        const float2 t2 = __fmul2_rn(make_float2(v[4][r], v[4][r + 1]), n2);
+        const float2 a0 = __ffma2_rn(make_float2(ex2(t0.x), ex2(t0.y)), mm0, one2);
+        const float2 a1 = __fadd2_rn(make_float2(ex2(t1.x), ex2(t1.y)), one2);
+        const float2 a2 = __ffma2_rn(make_float2(ex2(t2.x), ex2(t2.y)), mm2, one2);
+        const float2 P0 = __fmul2_rn(__fmul2_rn(a1, a2), mm0);
+        const float2 P1 = __fmul2_rn(a0, a2);
+        const float2 P2 = __fmul2_rn(__fmul2_rn(a0, a1), mm2);
+        const float2 Dn = __fadd2_rn(__fadd2_rn(P0, P1), P2);
+        bad |= (__float_as_int(Dn.x) > g.thr[r]) | (__float_as_int(Dn.y) > g.thr[r + 1]);
+        const float2 bx = __fmul2_rn(make_float2(v[0][r], v[0][r + 1]), make_float2(v[5][r], v[5][r + 1]));
+        W.P0[r] = P0.x; W.P0[r + 1] = P0.y;
+        W.P1[r] = P1.x; W.P1[r + 1] = P1.y;
+        W.P2[r] = P2.x; W.P2[r + 1] = P2.y;
+        W.rD[r] = rcp(Dn.x); W.rD[r + 1] = rcp(Dn.y);
+        W.bx[r] = bx.x; W.bx[r + 1] = bx.y;
+        W.uu[r] = v[1][r]; W.uu[r + 1] = v[1][r + 1];
+    }
+    if (R % 2) {
+        const int r = R - 1;
+        const float a0 = fmaf(ex2(v[2][r] * nl2e), g.m0[r], 1.0f);
+        const float a1 = ex2(v[3][r] * nl2e) + 1.0f;
+        const float a2 = fmaf(ex2(v[4][r] * nl2e), g.m2[r], 1.0f);
+        const float P0 = a1 * a2 * g.m0[r];
+        const float P1 = a0 * a2;
+        const float P2 = a0 * a1 * g.m2[r];
+        const float Dn = (P0 + P1) + P2;
+        bad |= __float_as_int(Dn) > g.thr[r];
+        W.P0[r] = P0;
+        W.P1[r] = P1;
+        W.P2[r] = P2;
+        W.rD[r] = rcp(Dn);
+        W.bx[r] = v[0][r] * v[5][r];
+        W.uu[r] = v[1][r];
+    }
+    return bad;
+}
+
+// Where the staged raw inputs of a line sit: element (t, r) is at
+// base[t] + off[r].
+template <int R>
+struct LineAddr {
+    const unsigned char *base[kTensors];
+    int off[R];
+};
+
+// Plain-form terms of one line (rare path): the normalised weights go in
+// P0..P2 with rD = 1, so the update is the same for both forms.  Same
+// arithmetic as the fast form's exponentials and reciprocals, without
+// products: sigmoid(z) = 1 / (1 + 2^(-z log2 e)) saturates to 0 or 1 instead
+// of overflowing, and the clamp of the local sum is explicit.
+template <int R>
+__device__ __forceinline__ void line_weights_plain_v(const float (&v)[kTensors][R], const LaneGeom<R> &g,
+                                                     LineW<R> &W) {
+    constexpr float nl2e = -1.4426950408889634f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const float s0 = rcp(1.0f + ex2(v[2][r] * nl2e)) * g.m0[r];
+        const float s1 = rcp(1.0f + ex2(v[3][r] * nl2e));
+        const float s2 = rcp(1.0f + ex2(v[4][r] * nl2e)) * g.m2[r];
+        const float iS = rcp(fmaxf((s0 + s1) + s2, 1e-6f));
+        W.P0[r] = s0 * iS;
+        W.P1[r] = s1 * iS;
+        W.P2[r] = s2 * iS;
+        W.rD[r] = 1.0f;
+        W.bx[r] = v[0][r] * v[5][r];
+        W.uu[r] = v[1][r];
+    }
+}
+
+template <typename T, int R>
+__device__ __forceinline__ void line_weights_plain(const LineAddr<R> &a, const LaneGeom<R> &g,
+                                                   LineW<R> &W) {
+    float v[kTensors][R];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t) v[t][r] = sload<T>(a.base[t] + a.off[r]);
+    line_weights_plain_v<R>(v, g, W);
+}
+
+// Column of output position j in a staged output row: bit 0 of j is flipped
+// in every other 32-column block, so that the row lanes' atomics on the
+// even (odd) positions 2l (2l+1) of a 64-position block hit 32 banks.
+__device__ __forceinline__ int ycol(int j) { return j ^ ((j >> 5) & 1); }
+
+// One step of the recurrence: h <- (sum_k P_k h(q+k-1)) / D + lambda x.  The
+// terms that need a neighbour lane's value (from the shuffles) come last.
+template <int R>
+__device__ __forceinline__ void recur(float (&h)[R], const LineW<R> &W) {
+    const float hl = __shfl_up_sync(0xffffffffu, h[R - 1], 1);
+    const float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
+    float hn[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float N = W.P1[r] * h[r];
+        if (r > 0) N = fmaf(W.P0[r], h[r - 1], N);
+        if (r < R - 1) N = fmaf(W.P2[r], h[r + 1], N);
+        if (r == 0) N = fmaf(W.P0[r], hl, N);
+        if (r == R - 1) N = fmaf(W.P2[r], hr, N);
+        hn[r] = fmaf(N, W.rD[r], W.bx[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) h[r] = hn[r];
+}
+
+// ---------------------------------------------------------------------------
+// Row lines (directions 0 and 1).
+// ---------------------------------------------------------------------------
+template <typename T, int R, bool FWD, int MODE>
+struct RowScan {
+    static constexpr int es = sizeof(T);
+    static constexpr int NP = R / 2;            // blocks of position pairs
+    static constexpr bool kSingle = (R % 2) != 0;
+    // raw words of one line per tensor: bf16 pairs share a 32-bit word
+    static constexpr int kWords = es == 2 ? NP + (kSingle ? 1 : 0) : R;
+    using Raw = uint32_t[kTensors][kWords];
+    static constexpr int kPrefetchAhead = 16;   // lines between an L2 prefetch and its use
+    static constexpr int kPrefetchLines = 8;    // lines per prefetch
+
+    const DirParams &p;
+    const int lane, D;
+    const int L, nch;
+    int total_chunks;
+    LaneGeom<R> g;
+    int eo[kWords];     // element offset (in a row) of each raw word, clamped into the row
+    int cs[R];          // output column of each position in the staged output plane
+    const char *gp[kTensors];   // the current item's planes
+    int item_k;                 // index of the current item among this CTA's items
+
+    __device__ static int pos(int lane, int r) {
+        return r < 2 * NP ? 64 * (r / 2) + 2 * lane + (r & 1) : 64 * NP + lane;
+    }
+
+    __device__ RowScan(const DirParams &p_, unsigned char *, int lane_, int d)
+        : p(p_), lane(lane_), D(d), L(p_.H), nch(1), total_chunks(0), item_k(0) {
+        const int W = p_.W;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = pos(lane_, r);
+            g.valid[r] = q < W;
+            g.m0[r] = q > 0 ? 1.0f : 0.0f;
+            g.m2[r] = q + 1 < W ? 1.0f : 0.0f;
+            g.thr[r] = __float_as_int((q > 0 && q + 1 < W) ? 1e11f : 1e5f);
+            cs[r] = q ^ ((q >> 5) & 1);
+        }
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) {
+            if (es == 2) {
+                // a pair word covers positions (q, q+1), q even; W is even
+                const int q = k < NP ? 64 * k + 2 * lane : 64 * NP + lane;
+                eo[k] = k < NP ? min(q, W - 2) : min(q, W - 1);
+            } else {
+                eo[k] = min(pos(lane_, k), W - 1);
             }
-            int hi;
-            chunk(c, lo, hi);
-            nl = hi - lo;
+        }
+    }
+
+    __device__ __forceinline__ void set_item(int k) {
+        item_k = k;
+        const int item = blockIdx.x + k * gridDim.x;
+        const int plane = item / p.bands;
+        const int b = plane / p.Cc, ch = plane - b * p.Cc;
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t) gp[t] = dir_tensor(p, t) + dir_plane(p, b, ch, D, t) * es;
+    }
+
+    __device__ __forceinline__ int row_of(int s) const { return FWD ? s : L - 1 - s; }
+
+    // Raw words of scan line s (global loads, L2-resident after the prefetch).
+    __device__ __forceinline__ void load(int s, Raw &w) const {
+        const int base = row_of(s) * p.W;
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) {
+            const int idx = base + eo[k];
 #pragma unroll
             for (int t = 0; t < kTensors; ++t) {
-                sp[t] = slot_ptr(stage, t);
-                shift[t] = ROW ? shifts[stage * 8 + t] : 0;
+                if (es == 2 && k < NP) w[t][k] = __ldg(reinterpret_cast<const unsigned int *>(gp[t]) + (idx >> 1));
+                else if (es == 2) w[t][k] = __ldg(reinterpret_cast<const unsigned short *>(gp[t]) + idx);
+                else w[t][k] = __ldg(reinterpret_cast<const unsigned int *>(gp[t]) + idx);
             }
-        };
+        }
+    }
 
-        // Iteration s (from -1) finishes line s and prepares line s+1: the
-        // rare plain form of line s, the chunk change, then one straight block
-        // with the weights of line s+1 and the recurrence of line s, then the
-        // outputs of line s.  tt is the scan-order index of line s in its chunk.
-        int c = 0, tt = -1;
-        enter_chunk(0);
-        LineW<R> Wc;
-        Wc.bad = false;
-        int cur = 0;
+    __device__ __forceinline__ static void unpack(const Raw &w, float (&v)[kTensors][R]) {
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t)
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (es == 4) v[t][r] = __uint_as_float(w[t][r]);
+                else if (r < 2 * NP) v[t][r] = __uint_as_float((r & 1) ? (w[t][r / 2] & 0xffff0000u) : (w[t][r / 2] << 16));
+                else v[t][r] = __uint_as_float(w[t][NP] << 16);
+            }
+    }
+
+    // L2 prefetch (bulk prefetch, TMA engine) of lines [s0, s0 + kPrefetchLines)
+    // of the warp's line stream, which continues into its next item.
+    __device__ __forceinline__ void prefetch(int s0) const {
+        if (lane >= kTensors) return;
+        int k = item_k, s = s0;
+        while (s >= L) { s -= L; ++k; }
+        const int item = blockIdx.x + k * gridDim.x;
+        if (item >= p.n_items) return;
+        const int plane = item / p.bands;
+        const int b = plane / p.Cc, ch = plane - b * p.Cc;
+        const int t = lane;
+        const int n = min(kPrefetchLines, L - s);
+        const int r0 = FWD ? s : L - s - n;
+        const char *base = dir_tensor(p, t);
+        const unsigned long long end = dir_tensor_bytes(p, t);
+        unsigned long long a = (dir_plane(p, b, ch, D, t) + static_cast<size_t>(r0) * p.W) * es;
+        unsigned long long e = a + static_cast<unsigned long long>(n) * p.W * es;
+        a &= ~15ull;
+        e = (e + 15) & ~15ull;
+        if (e > end) e = end & ~15ull;
+        if (e > a) prefetch_l2(base + a, static_cast<uint32_t>(e - a));
+    }
+
+    __device__ __forceinline__ void plain_line(int s, LineW<R> &W) const {
+        Raw w;
+        load(s, w);
+        float v[kTensors][R];
+        unpack(w, v);
+        line_weights_plain_v<R>(v, g, W);
+    }
+
+    // Gated output of the step's row into the output plane / band / global.
+    __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int row, uint32_t ysa,
+                                         float *yg, int band_lo, int band_hi) const {
+        const bool in = MODE != kYBanded || (row >= band_lo && row < band_hi);
+        const uint32_t yl = ysa + 4u * static_cast<uint32_t>((row - band_lo) * p.y_pitch);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float cy = W.uu[r] * h[r];
+            if (MODE == kYGlobal) {
+                if (g.valid[r]) atomicAdd(yg + static_cast<size_t>(row) * p.W + pos(lane, r), cy);
+            } else {
+                red_add_shared_if(yl + 4u * cs[r], cy, g.valid[r] && in);
+            }
+        }
+    }
+
+    // One step of the recurrence with this lane layout: positions 2l, 2l+1
+    // of each 64-position block and 64 NP + l; the neighbours across lanes
+    // (and across blocks, between lanes 31 and 0) come from shuffles.
+    __device__ __forceinline__ void recur_rows(float (&h)[R], const LineW<R> &W) const {
+        float left[R], right[R];
+#pragma unroll
+        for (int p2 = 0; p2 < NP; ++p2) {
+            const int a = 2 * p2, b = 2 * p2 + 1;
+            // left of the even position: lane-1's odd one; lane 0 takes the
+            // previous block's last position from lane 31
+            const float sendl = (p2 > 0 && lane == 31) ? h[a - 1] : h[b];
+            left[a] = __shfl_sync(0xffffffffu, sendl, (lane + 31) & 31);
+            left[b] = h[a];
+            // right of the odd position: lane+1's even one; lane 31 takes
+            // the next block's first position from lane 0
+            const int nxt = b + 1 < R ? b + 1 : b;
+            const float sendr = (b + 1 < R && lane == 0) ? h[nxt] : h[a];
+            right[b] = __shfl_sync(0xffffffffu, sendr, (lane + 1) & 31);
+            right[a] = h[b];
+        }
+        if (kSingle) {
+            const int s1 = R - 1;
+            const float sendl = (NP > 0 && lane == 31) ? h[s1 > 0 ? s1 - 1 : 0] : h[s1];
+            left[s1] = __shfl_sync(0xffffffffu, sendl, (lane + 31) & 31);
+            right[s1] = __shfl_down_sync(0xffffffffu, h[s1], 1);
+        }
+        float hn[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float N = W.P1[r] * h[r];
+            N = fmaf(W.P0[r], left[r], N);
+            N = fmaf(W.P2[r], right[r], N);
+            hn[r] = fmaf(N, W.rD[r], W.bx[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) h[r] = hn[r];
+    }
+
+    // Step s (J = s mod 2): the plain form if line s was flagged, the update
+    // of line s, the weights of line s+1 (its raw words arrived two steps
+    // ago), the loads of line s+3 into the freed buffer, the outputs.
+    template <int J, bool CHECK>
+    __device__ __forceinline__ void step(int s, float (&h)[R], LineW<R> (&Wb)[2], bool (&bad)[2],
+                                         Raw (&rb)[2], uint32_t ysa, float *yg, int band_lo, int band_hi) {
+        LineW<R> &Wc = Wb[J];
+        if (__any_sync(0xffffffffu, bad[J])) plain_line(s, Wc);
+        recur_rows(h, Wc);
+        if (!CHECK || s + 1 < L) {
+            float v[kTensors][R];
+            unpack(rb[J ^ 1], v);
+            bad[J ^ 1] = line_weights(v, g, Wb[J ^ 1]);
+            if (!CHECK || s + 3 < L) load(s + 3, rb[J ^ 1]);
+        }
+        emit(h, Wc, row_of(s), ysa, yg, band_lo, band_hi);
+    }
+
+    // Run every line of the CTA's k-th item.
+    __device__ void run_item(int k, float *ys, float *yg, int band_lo, int band_hi) {
+        const uint32_t ysa = smem_u32(ys);
+        set_item(k);
+        if (k == 0) {
+            for (int s0 = 0; s0 < kPrefetchAhead; s0 += kPrefetchLines) prefetch(s0);
+        }
+        float h[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) h[r] = 0.0f;
+        LineW<R> Wb[2];
+        bool bad[2];
+        Raw rb[2];
+        load(0, rb[0]);
+        if (L > 1) load(1, rb[1]);
+        {
+            float v[kTensors][R];
+            unpack(rb[0], v);
+            bad[0] = line_weights(v, g, Wb[0]);
+        }
+        if (L > 2) load(2, rb[0]);
+        int s = 0;
 #pragma unroll 1
-        for (int s = -1; s < L; ++s) {
-            float hl = __shfl_up_sync(0xffffffffu, hs[R - 1], 1);
-            float hr = __shfl_down_sync(0xffffffffu, hs[0], 1);
-            float hp[R];
-            const bool plain = s >= 0 && __any_sync(0xffffffffu, Wc.bad);
-            if (plain) plain_line(sp, shift, fwd ? tt : nl - 1 - tt, hs, hl, hr, hp);
-            int tt1 = tt + 1;
-            if (s + 1 < L && tt1 == nl) {
-                ++g;
-                ++c;
-                tt1 = 0;
-                enter_chunk(c);
+        for (; s + 4 < L; s += 2) {
+            if ((s & (kPrefetchLines - 1)) == 0) prefetch(s + kPrefetchAhead);
+            step<0, false>(s, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
+            step<1, false>(s + 1, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
+        }
+        // the last lines
+#pragma unroll 1
+        for (; s < L; s += 2) {
+            if ((s & (kPrefetchLines - 1)) == 0) prefetch(s + kPrefetchAhead);
+            step<0, true>(s, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
+            if (s + 1 < L) step<1, true>(s + 1, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Column lines (directions 2 and 3).
+// ---------------------------------------------------------------------------
+template <typename T, int R, bool FWD, int MODE>
+struct ColScan {
+    static constexpr int es = sizeof(T);
+    static constexpr int NS = kColStages;
+    static constexpr int CH = kColStrip / es;   // columns (steps) per chunk: 8 bf16, 4 fp32
+    static constexpr int NB = CH / 4;           // 4-step bodies per chunk: 2 bf16, 1 fp32
+    // Two consecutive columns of a strip row are one 32-bit (bf16) or 64-bit
+    // (fp32) word; a body's two word sets cover its four columns.
+    using Pair = typename std::conditional<es == 2, uint32_t, uint2>::type;
+    using PairSet = Pair[kTensors][R];
+    static constexpr int kCopyRows = 32 / 4;    // grid rows per copy instruction (4 lanes per row)
+
+    const DirParams &p;
+    const int lane, D;
+    unsigned char *const ring;
+    const int L, nch;
+    int total_chunks;
+    LaneGeom<R> g;
+    int rowq[R];        // byte offset of strip row q_r in a stage (row 0 when q_r >= H)
+    int fsw[R];         // word swizzle of that strip row (see swz)
+    bool inb[R];        // q_r is an output row of the current item
+    uint32_t ya[R];     // shared address of column 0 of its output row
+    int issue_item;
+    const char **gtab;  // [kTensors] planes of the item being issued (shared memory)
+
+    __device__ ColScan(const DirParams &p_, unsigned char *smem, int lane_, int d)
+        : p(p_), lane(lane_), D(d),
+          ring(smem + (d == 2 ? p_.ring[2] : p_.ring[3])),
+          L(p_.W), nch((p_.W + kColStrip / static_cast<int>(sizeof(T)) - 1) /
+                       (kColStrip / static_cast<int>(sizeof(T)))),
+          total_chunks(0), issue_item(-1),
+          gtab(reinterpret_cast<const char **>(smem + p_.bar_off + 128 + 64 * (d - 2))) {
+        g.init(lane_, p_.H);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = lane_ * R + r < p_.H ? lane_ * R + r : 0;
+            rowq[r] = q * kColPitch;
+            fsw[r] = swz(q);
+        }
+    }
+
+    // bf16 strips are read one 32-bit word per lane (all 32 lanes in one
+    // wavefront): lanes l and l+16 read rows 48 apart (R = 3), whose 104-byte
+    // pitches put them on the same bank, so bit 0 of the word index within a
+    // strip row is flipped on every other band of 16R rows.  fp32 strips are
+    // read 64 bits per lane, half a warp per wavefront, already conflict-free.
+    __device__ __forceinline__ static int swz(int q) { return es == 2 ? (q / (16 * R)) & 1 : 0; }
+
+    // Lowest column of chunk c (chunks are numbered in scan order).
+    __device__ __forceinline__ int chunk_lo(int c) const { return FWD ? c * CH : L - CH - c * CH; }
+
+    __device__ __forceinline__ unsigned char *stage_ptr(int gi) const {
+        return ring + (gi % NS) * p.stage_col;
+    }
+
+    // The warp copies the strip: lane (i0, w) = (lane / 4, lane % 4) moves
+    // word w of grid rows i0, i0 + 8, ... of every tensor (4 lanes cover
+    // one row's 16 bytes, so a copy instruction reads 8 rows).
+    template <bool FULL>
+    __device__ __forceinline__ void copy_strip(uint32_t sb, int lo) const {
+        const char *gt[kTensors];
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t) gt[t] = gtab[t];
+        const int w = lane & 3, i0 = lane >> 2;
+        if (!FULL) {
+            const int col = lo + w * (4 / es);
+            if (col < 0 || col + 4 / es > L) return;
+        }
+        // right-to-left scans store the words of a strip row reversed
+        const int dw = FWD ? w : 3 - w;
+        const int rowstep = kCopyRows * p.W * es;
+        int src_off = (i0 * p.W + lo) * es + 4 * w;
+        uint32_t drow = sb + static_cast<uint32_t>(i0 * kColPitch);
+#pragma unroll 1
+        for (int row = i0; row < p.H; row += kCopyRows) {
+            const uint32_t dst = drow + 4u * static_cast<uint32_t>(dw ^ swz(row));
+#pragma unroll
+            for (int t = 0; t < kTensors; ++t) cp_async_4(dst + 16 * t, gt[t] + src_off);
+            src_off += rowstep;
+            drow += kCopyRows * kColPitch;
+        }
+    }
+
+    // Issue (and commit as one group) the warp's copies of chunk gi.  Every
+    // read of the stage it overwrites (chunk gi-2) is complete: the values
+    // were consumed before this point.
+    __device__ __forceinline__ void issue(int gi) {
+        __syncwarp();
+        if (gi < total_chunks) {
+            const int kk = gi / nch;
+            const int c = gi - kk * nch;
+            const int item = blockIdx.x + kk * gridDim.x;
+            if (item != issue_item) {
+                issue_item = item;
+                const int plane = item / p.bands;
+                const int b = plane / p.Cc, ch = plane - b * p.Cc;
+                if (lane < kTensors) gtab[lane] = dir_tensor(p, lane) + dir_plane(p, b, ch, D, lane) * es;
+                __syncwarp();
             }
-            LineW<R> Wn;
-            weights(sp, shift, fwd ? tt1 : nl - 1 - tt1, m0, m2, ithr, valid, Wn);
-            float hn[R];
+            const int lo = chunk_lo(c);
+            const uint32_t sb = smem_u32(stage_ptr(gi));
+            if (lo >= 0 && lo + CH <= L) copy_strip<true>(sb, lo);
+            else copy_strip<false>(sb, lo);
+        }
+        cp_async_commit();
+    }
+
+    // Wait until at most N of the warp's copy groups are in flight; rows are
+    // copied by other lanes than the ones that read them.
+    template <int N>
+    __device__ __forceinline__ void wait() const {
+        cp_async_wait<N>();
+        __syncwarp();
+    }
+
+    // Word set of the column pair `pidx` (0..3 in scan order within a strip
+    // row; always even or always odd at a given call site) of a stage.
+    __device__ __forceinline__ void load_pair(const unsigned char *sp, int pidx, PairSet &w) const {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            // word (pidx ^ fsw) of the bf16 strip row; fp32 pairs are 8 bytes
+            const int off = es == 2 ? rowq[r] + 4 * pidx + ((pidx & 1) ? -4 : 4) * fsw[r]
+                                    : rowq[r] + 8 * pidx;
+#pragma unroll
+            for (int t = 0; t < kTensors; ++t)
+                w[t][r] = *reinterpret_cast<const Pair *>(sp + off + 16 * t);
+        }
+    }
+
+    // Column K (0 or 1, scan order) of a word set as floats.
+    template <int K>
+    __device__ __forceinline__ static void unpack(const PairSet &w, float (&v)[kTensors][R]) {
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t)
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float left = r > 0 ? hs[r - 1] : hl;
-                const float right = r < R - 1 ? hs[r + 1] : hr;
-                float N = Wc.P0[r] * left;
-                N = fmaf(Wc.P1[r], hs[r], N);
-                N = fmaf(Wc.P2[r], right, N);
-                hn[r] = fmaf(N, Wc.rD[r], Wc.bx[r]);
-                if (plain) hn[r] = hp[r];
-            }
-            float uu[R];
-#pragma unroll
-            for (int r = 0; r < R; ++r) uu[r] = Wc.uu[r];
-            const int line = cur;   // grid line of step s
-            Wc = Wn;
-            tt = tt1;
-            cur = fwd ? lo + tt : lo + nl - 1 - tt;
-            if (s < 0) continue;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                hs[r] = valid[r] ? hn[r] : 0.0f;
-                const float cy = uu[r] * hs[r];
-                const int q = lane * R + r;
-                if (MODE == kYGlobal) {
-                    if (valid[r]) {
-                        if (ROW) atomicAdd(yg + static_cast<size_t>(line) * p.W + q, cy);
-                        else atomicAdd(yg + static_cast<size_t>(q) * p.W + line, cy);
-                    }
-                } else if (ROW) {
-                    const bool in = MODE != kYBanded || (line >= band_lo && line < band_hi);
-                    red_add_shared_if(ysa + 4u * ((line - band_lo) * p.y_pitch + q), cy, valid[r] && in);
+                if constexpr (es == 4) {
+                    v[t][r] = __uint_as_float(K == 0 ? w[t][r].x : w[t][r].y);
                 } else {
-                    red_add_shared_if(ysa + 4u * ((q - band_lo) * p.y_pitch + line), cy, inband[r]);
+                    // a word holds columns (2m, 2m+1); reversed sweeps meet the odd one first
+                    const bool hi = FWD ? (K & 1) : !(K & 1);
+                    v[t][r] = __uint_as_float(hi ? (w[t][r] & 0xffff0000u) : (w[t][r] << 16));
+                }
+            }
+    }
+
+    // Byte offset, within a strip row's 16-byte piece, of the chunk's step k
+    // for position r (swizzled word, then the bf16 half).
+    __device__ __forceinline__ int step_byte(int k, int r) const {
+        return es == 4 ? 4 * k : 4 * ((k / 2) ^ fsw[r]) + 2 * (FWD ? (k & 1) : 1 - (k & 1));
+    }
+
+    // Step k of the staged chunk gi, read from shared memory.
+    __device__ __forceinline__ void reload(int gi, int k, float (&v)[kTensors][R]) const {
+        const unsigned char *sp = stage_ptr(gi);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int off = rowq[r] + step_byte(k, r);
+#pragma unroll
+            for (int t = 0; t < kTensors; ++t) v[t][r] = sload<T>(sp + off + 16 * t);
+        }
+    }
+
+    __device__ __forceinline__ void plain(int gi, int k, LineW<R> &W) const {
+        LineAddr<R> a;
+        const unsigned char *sp = stage_ptr(gi);
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t) a.base[t] = sp + 16 * t;
+#pragma unroll
+        for (int r = 0; r < R; ++r) a.off[r] = rowq[r] + step_byte(k, r);
+        line_weights_plain<T, R>(a, g, W);
+    }
+
+    __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int col, float *yg) const {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float cy = W.uu[r] * h[r];
+            if (MODE == kYGlobal) {
+                if (g.valid[r]) atomicAdd(yg + static_cast<size_t>(lane * R + r) * p.W + col, cy);
+            } else {
+                red_add_shared_if(ya[r] + 4u * ycol(col), cy, inb[r]);
+            }
+        }
+    }
+
+    // Step J of body b of the full chunk c (launch chunk number gi): steps
+    // 0-1 read word set A, steps 2-3 word set B.  B is loaded by step 0; the
+    // next body's A by step 2 (from the next chunk, waited for here, when b
+    // is the chunk's last body); `last` when chunk c ends the item.
+    template <int J>
+    __device__ __forceinline__ void bstep(int gi, int c, int b, bool last, float (&h)[R],
+                                          LineW<R> (&Wb)[2], bool (&bad)[2], PairSet &A, PairSet &B,
+                                          float *yg) {
+        LineW<R> &Wc = Wb[J & 1];
+        const int k = 4 * b + J;   // step within the chunk
+        if (__any_sync(0xffffffffu, bad[J & 1])) plain(gi, k, Wc);
+        recur(h, Wc);
+        const bool more = b + 1 < NB || !last;   // a step follows this body's last
+        if (J == 0) load_pair(stage_ptr(gi), 2 * b + 1, B);
+        if (J == 2 && more) {
+            if (b + 1 < NB) {
+                load_pair(stage_ptr(gi), 2 * b + 2, A);
+            } else {
+                wait<0>();               // chunk gi+1 (issued when chunk gi was entered)
+                load_pair(stage_ptr(gi + 1), 0, A);
+            }
+        }
+        // weights of the next step
+        if (J < 3 || more) {
+            float v[kTensors][R];
+            if (J == 0) unpack<1>(A, v);
+            else if (J == 1) unpack<0>(B, v);
+            else if (J == 2) unpack<1>(B, v);
+            else unpack<0>(A, v);
+            bad[(J + 1) & 1] = line_weights(v, g, Wb[(J + 1) & 1]);
+        }
+        emit(h, Wc, FWD ? c * CH + k : L - 1 - c * CH - k, yg);
+    }
+
+    // Step k of the item's last, partial chunk (n < CH steps), reading each
+    // column from shared memory; J = k mod 2 picks the weight set.
+    template <int J>
+    __device__ __forceinline__ void pstep(int gi, int c, int k, int n, float (&h)[R], LineW<R> (&Wb)[2],
+                                          bool (&bad)[2], float *yg) {
+        LineW<R> &Wc = Wb[J];
+        if (__any_sync(0xffffffffu, bad[J])) plain(gi, k, Wc);
+        recur(h, Wc);
+        if (k + 1 < n) {
+            float v[kTensors][R];
+            reload(gi, k + 1, v);
+            bad[J ^ 1] = line_weights(v, g, Wb[J ^ 1]);
+        }
+        emit(h, Wc, FWD ? c * CH + k : L - 1 - c * CH - k, yg);
+    }
+
+    // Run every column of the item whose first chunk is g0.
+    __device__ void run_item(int g0, float *ys, float *yg, int band_lo, int band_hi) {
+        const uint32_t ysa = smem_u32(ys);
+        float h[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            h[r] = 0.0f;
+            const int q = lane * R + r;
+            inb[r] = g.valid[r] && (MODE != kYBanded || (q >= band_lo && q < band_hi));
+            ya[r] = ysa + 4u * static_cast<uint32_t>((inb[r] ? q - band_lo : 0) * p.y_pitch);
+        }
+        LineW<R> Wb[2];
+        bool bad[2];
+        PairSet A, B;
+        const int nfull = L / CH;
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            const int gi = g0 + c;
+            // entering chunk gi: the stage of chunk gi-1 is free for gi+1
+            issue(gi + 1);
+            if (c == 0) {
+                // the item's first chunk: wait for it, weights of step 0
+                wait<1>();
+                float v[kTensors][R];
+                if (nfull > 0) {
+                    load_pair(stage_ptr(gi), 0, A);
+                    unpack<0>(A, v);
+                } else {
+                    reload(gi, 0, v);
+                }
+                bad[0] = line_weights(v, g, Wb[0]);
+            }
+            if (c < nfull) {
+                const bool last = c + 1 == nch;
+#pragma unroll 1
+                for (int b = 0; b < NB; ++b) {
+                    bstep<0>(gi, c, b, last, h, Wb, bad, A, B, yg);
+                    bstep<1>(gi, c, b, last, h, Wb, bad, A, B, yg);
+                    bstep<2>(gi, c, b, last, h, Wb, bad, A, B, yg);
+                    bstep<3>(gi, c, b, last, h, Wb, bad, A, B, yg);
+                }
+            } else {
+                const int n = L - c * CH;
+#pragma unroll 1
+                for (int k = 0; k < n; k += 2) {
+                    pstep<0>(gi, c, k, n, h, Wb, bad, yg);
+                    if (k + 1 < n) pstep<1>(gi, c, k + 1, n, h, Wb, bad, yg);
                 }
             }
         }
-        ++g;   // the last chunk of the item is done
     }
 };
 
@@ -456,25 +793,23 @@ __device__ __forceinline__ void dir_barrier() {
     asm volatile("bar.sync 1, %0;" ::"n"(kDirThreads) : "memory");
 }
 
-// The whole kernel seen from the warp that runs direction D (row lines when
-// ROW); only that orientation's state is live in its registers, and the two
-// directions of an orientation share one code path.
-template <typename T, int R, bool ROW, int MODE>
+// The whole kernel seen from the warp that runs direction D.
+template <typename T, int R, bool ROW, bool FWD, int MODE>
 __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem, int warp, int lane, int D) {
     float *ys = reinterpret_cast<float *>(smem);   // output plane or band, fp32 [rows][y_pitch]
     const int YP = p.y_pitch;
     const bool active = (p.dirs >> D) & 1;
     const int n_my = blockIdx.x < p.n_items ? (p.n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    DirWarp<T, R, ROW, MODE> w(p, smem, lane, D);
-    constexpr int NS = kDirStages;
-    const int total = active ? n_my * w.nch : 0;
-    for (int s = 0; s < NS - 1; ++s) {
-        if (s < total) w.issue(blockIdx.x, s, s);
-        else if (!ROW) cp_async_commit();
+    using Scan = typename std::conditional<ROW, RowScan<T, R, FWD, MODE>, ColScan<T, R, FWD, MODE>>::type;
+    Scan sc(p, smem, lane, D);
+    const int total = active ? n_my * sc.nch : 0;
+    sc.total_chunks = total;
+    // column lines: the first chunk; each chunk entered later issues the next
+    if constexpr (!ROW) {
+        if (active) sc.issue(0);
     }
 
-    int g = 0;
     for (int k = 0; k < n_my; ++k) {
         const int item = blockIdx.x + k * gridDim.x;
         const int plane = item / p.bands;
@@ -487,42 +822,47 @@ __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem
             for (int e = threadIdx.x; e < p.H * p.W; e += kDirThreads) yg[e] = 0.0f;
             dir_barrier();
         }
-        if (active) w.run_item(item, g, total, ys, yg, band_lo, band_hi);
+        if (active) sc.run_item(ROW ? k : k * sc.nch, ys, yg, band_lo, band_hi);
         dir_barrier();
         if (MODE != kYGlobal) {
             // write the band out once (converted) and clear it for the next item
             T *outp = static_cast<T *>(p.out) + static_cast<size_t>(plane) * p.H * p.W +
                       static_cast<size_t>(band_lo) * p.W;
             for (int i = warp; i < band_hi - band_lo; i += 4) {
-                float *yrow = ys + i * YP;
+                float *yr = ys + i * YP;
                 T *orow = outp + static_cast<size_t>(i) * p.W;
                 for (int j = lane; j < p.W; j += 32) {
-                    orow[j] = from_f<T>(yrow[j]);
-                    yrow[j] = 0.0f;
+                    const int yc = ycol(j);
+                    orow[j] = from_f<T>(yr[yc]);
+                    yr[yc] = 0.0f;
                 }
             }
             dir_barrier();
         }
     }
-    cp_async_wait<0>();
+    if (!ROW) cp_async_wait<0>();
 }
 
+// Lines of up to 96 positions keep three CTAs (12 warps) per SM: the
+// register budget is then 168 per thread.
 template <typename T, int R, int MODE>
-__global__ void __launch_bounds__(kDirThreads)
+__global__ void __launch_bounds__(kDirThreads, R <= 3 ? 3 : 2)
 prop2d_dir_kernel(const DirParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float *ys = reinterpret_cast<float *>(smem);
-    if (MODE != kYGlobal)
-        for (int e = threadIdx.x; e < p.band_rows * p.y_pitch; e += kDirThreads) ys[e] = 0.0f;
-    if (threadIdx.x == 0) {
-        // one arrival per tensor span of a row chunk
-        for (int i = 0; i < 2 * kDirStages; ++i) mbar_init(smem_u32(smem + p.bar_off) + 8 * i, kTensors);
-        mbar_init_fence();
+    // Zero the output plane and the rings: staged slots then never hold
+    // non-finite values, also where positions past a line's end read them.
+    {
+        uint4 *z = reinterpret_cast<uint4 *>(smem);
+        for (int e = threadIdx.x; e < p.bar_off / 16; e += kDirThreads) z[e] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    if (warp < 2) dir_role<T, R, true, MODE>(p, smem, warp, lane, warp);
-    else dir_role<T, R, false, MODE>(p, smem, warp, lane, warp);
+    switch (warp) {
+        case 0: dir_role<T, R, true, true, MODE>(p, smem, warp, lane, 0); break;
+        case 1: dir_role<T, R, true, false, MODE>(p, smem, warp, lane, 1); break;
+        case 2: dir_role<T, R, false, true, MODE>(p, smem, warp, lane, 2); break;
+        default: dir_role<T, R, false, false, MODE>(p, smem, warp, lane, 3); break;
+    }
 }
 
 }  // namespace gspn
