@@ -22,7 +22,10 @@ cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t 
     li.grid = static_cast<int>(grid);
     li.block = gspn::kDirThreads;
     li.smem = pl.smem;
-    li.path = MODE == gspn::kYGlobal ? "dir-yglobal" : MODE == gspn::kYBanded ? "dir-banded" : "dir";
+    li.path = MODE == gspn::kYGlobal   ? "dir-yglobal"
+              : MODE == gspn::kYBanded ? "dir-banded"
+              : MODE == gspn::kYShared ? "dir-shared"
+                                       : "dir";
     return cudaGetLastError();
 }
 

@@ -52,30 +52,38 @@ cudaError_t device_props(DeviceProps &dp) {
 }
 
 // Shared-memory plan for output mode `mode` so that one CTA fits `cap`
-// bytes.  Output modes: 0, the fp32 output plane in shared memory; 1, fp32
-// outputs accumulated in global memory (L2 atomics); 2, row bands of the
-// output plane in shared memory (the scans are rerun per band).  Layout:
-// output plane or band, the column rings of the enabled column directions,
-// then the column warps' plane-pointer tables.
+// bytes.  Output modes: 0, fp32 output planes in shared memory (one for the
+// row directions, one for the column directions); 1, fp32 outputs
+// accumulated in global memory (L2 atomics); 2, row bands of the two planes
+// in shared memory (the scans are rerun per band); 3, one fp32 plane in
+// shared memory that all directions add into with shared-memory atomics.  Layout: row plane or
+// band, column plane or band, the column rings of the enabled column
+// directions, then the column warps' plane-pointer tables.
 bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
     const int n_col = ((dirs >> 2) & 1) + ((dirs >> 3) & 1);
-    // odd pitch above every swizzled column index (see ycol)
+    // odd pitch above every swizzled column index (see ycol), whose last
+    // column is a dummy written by row lanes past the end of a row
     const int YP = (W % 2 == 0) ? W + 1 : W + 2;
     const int stage_col = round_up(H * gspn::kColPitch, 16);
     const int col_ring = gspn::kColStages * stage_col;
     const int rings = n_col * col_ring + gspn::kDirBarBytes;
-    int band_rows = H, y_bytes = 0;
-    if (mode == 0) {
-        y_bytes = round_up(H * YP * 4, 16);
+    const int n_planes = mode == 3 ? 1 : ((dirs & 3) ? 1 : 0) + ((dirs & 12) ? 1 : 0);
+    // a plane holds its rows plus one dummy row (written by the column lanes
+    // past the end of a column or outside the band)
+    int band_rows = H, plane_bytes = 0;
+    if (mode == 0 || mode == 3) {
+        plane_bytes = round_up((H + 1) * YP * 4, 16);
     } else if (mode == 2) {
-        if (cap - rings < YP * 4) return false;
-        band_rows = (cap - rings) / (YP * 4);
+        if (cap - rings < n_planes * 2 * YP * 4) return false;
+        band_rows = (cap - rings) / (n_planes * YP * 4) - 1;
         if (band_rows > H) band_rows = H;
-        y_bytes = round_up(band_rows * YP * 4, 16);
+        plane_bytes = round_up((band_rows + 1) * YP * 4, 16);
     }
+    const int y_bytes = n_planes * plane_bytes;
     if (y_bytes + rings > cap) return false;
     DirParams &p = pl.p;
     p.stage_col = stage_col;
+    p.ycol_off = (mode != 3 && (dirs & 3)) ? plane_bytes : 0;
     int off = y_bytes;
     for (int d = 0; d < 4; ++d) {
         if (d < 2 || !((dirs >> d) & 1)) { p.ring[d] = -1; continue; }
@@ -88,6 +96,7 @@ bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
     p.bands = (H + band_rows - 1) / band_rows;
     pl.smem = y_bytes + rings;
     pl.y_global = mode == 1;
+    pl.y_shared = mode == 3;
     return true;
 }
 
@@ -162,14 +171,17 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
         DirPlan pl;
         pl.p.x = x; pl.p.lam = lambda; pl.p.wl = wlogit; pl.p.u = u; pl.p.out = out;
         pl.p.B = B; pl.p.Cc = Cc; pl.p.H = H; pl.p.W = W; pl.p.dirs = dirs; pl.p.share_w = share_w;
-        // Output modes in order of preference (whole plane in shared memory,
-        // fp32 plane in global memory, bands: the last reruns the scans per
+        // Output modes in order of preference (the last reruns the scans per
         // band); within a mode, the most CTAs per SM that fit.
         const int caps[4] = {dp.smem_per_sm / 4 - 1024, dp.smem_per_sm / 3 - 1024,
                              dp.smem_per_sm / 2 - 1024, dp.smem_optin};
         bool fit = false;
-        for (int mode = 0; mode < 3 && !fit; ++mode) {
-            if (mode == 1 && es != 4) continue;
+        // two planes; then one plane with shared atomics (bf16) or global
+        // atomics (fp32); then bands
+        const int order[4] = {0, 3, 1, 2};
+        for (int oi = 0; oi < 4 && !fit; ++oi) {
+            const int mode = order[oi];
+            if ((mode == 1 && es != 4) || (mode == 3 && es != 2)) continue;
             for (int ci = 0; ci < 4 && !fit; ++ci) {
                 const int cap = caps[ci] < dp.smem_optin ? caps[ci] : dp.smem_optin;
                 fit = plan_dir_fit(pl, cap, H, W, dirs, mode);
@@ -188,8 +200,9 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
                       : banded    ? launch_dir_f32_banded(R, pl, dp, stream, g_last)
                                   : launch_dir_f32_smem(R, pl, dp, stream, g_last);
             } else {
-                err = banded ? launch_dir_bf16_banded(R, pl, dp, stream, g_last)
-                             : launch_dir_bf16_smem(R, pl, dp, stream, g_last);
+                err = pl.y_shared ? launch_dir_bf16_shared(R, pl, dp, stream, g_last)
+                      : banded    ? launch_dir_bf16_banded(R, pl, dp, stream, g_last)
+                                  : launch_dir_bf16_smem(R, pl, dp, stream, g_last);
             }
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }

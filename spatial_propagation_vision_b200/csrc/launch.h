@@ -25,6 +25,7 @@ struct DeviceProps {
 // Launch geometry of the direction kernel.
 struct DirPlan {
     bool y_global = false;
+    bool y_shared = false;   // one plane, shared-memory atomics
     int smem = 0;
     gspn::DirParams p{};
 };
@@ -38,6 +39,7 @@ cudaError_t launch_dir_f32_banded(int R, const DirPlan &pl, const DeviceProps &d
 cudaError_t launch_dir_f32_global(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_smem(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_banded(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_shared(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 
 // General kernel; `fits` is false when even one output row does not fit.
 cudaError_t launch_generic(const gspn::GenericParams &gp, bool bf16, const DeviceProps &dp,

@@ -67,6 +67,8 @@ constexpr int kDirBarBytes = 256;  // plane-pointer tables of the column warps
 constexpr int kYSmem = 0;     // whole fp32 output plane in shared memory
 constexpr int kYBanded = 1;   // a band of output rows in shared memory, scans rerun per band
 constexpr int kYGlobal = 2;   // fp32 output accumulated in global memory (L2 atomics)
+constexpr int kYShared = 3;   // one fp32 plane in shared memory for all four directions
+                              // (shared-memory atomics): planes too large for two
 
 struct DirParams {
     const void *x, *lam, *wl, *u;
@@ -76,6 +78,7 @@ struct DirParams {
     int stage_col;              // bytes per column ring stage
     int ring[4];                // byte offset of column direction d's ring (-1: none)
     int bar_off;                // byte offset of the column warps' plane-pointer tables
+    int ycol_off;               // byte offset of the column directions' output plane
     int y_pitch;                // floats per staged output row (odd, > every ycol(j), j < W)
     unsigned long long end_x, end_gate, end_wl;   // byte sizes of x, lambda/u, logits
     unsigned int *status;       // device status word (bounded waits that gave up)
@@ -84,6 +87,12 @@ struct DirParams {
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// Byte permutation of (x, 0): bf16 half of a word -> fp32 bits.
+__device__ __forceinline__ uint32_t prmt0(uint32_t x, uint32_t sel) {
+    uint32_t y;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(x), "r"(sel));
     return y;
 }
 __device__ __forceinline__ float rcp(float x) {
@@ -197,14 +206,6 @@ __device__ __forceinline__ bool line_weights(const float (&v)[kTensors][R], cons
     return bad;
 }
 
-// Where the staged raw inputs of a line sit: element (t, r) is at
-// base[t] + off[r].
-template <int R>
-struct LineAddr {
-    const unsigned char *base[kTensors];
-    int off[R];
-};
-
 // Plain-form terms of one line (rare path): the normalised weights go in
 // P0..P2 with rD = 1, so the update is the same for both forms.  Same
 // arithmetic as the fast form's exponentials and reciprocals, without
@@ -229,21 +230,40 @@ __device__ __forceinline__ void line_weights_plain_v(const float (&v)[kTensors][
     }
 }
 
-template <typename T, int R>
-__device__ __forceinline__ void line_weights_plain(const LineAddr<R> &a, const LaneGeom<R> &g,
-                                                   LineW<R> &W) {
-    float v[kTensors][R];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int t = 0; t < kTensors; ++t) v[t][r] = sload<T>(a.base[t] + a.off[r]);
-    line_weights_plain_v<R>(v, g, W);
+// Terms of one line from its raw inputs: the fast form, or the plain form
+// for the whole line (every lane) when some position is out of the fast
+// form's range.
+template <int R>
+__device__ __forceinline__ void line_terms(const float (&v)[kTensors][R], const LaneGeom<R> &g, LineW<R> &W) {
+    const bool bad = line_weights(v, g, W);
+    if (__any_sync(0xffffffffu, bad)) line_weights_plain_v<R>(v, g, W);
 }
 
 // Column of output position j in a staged output row: bit 0 of j is flipped
 // in every other 32-column block, so that the row lanes' atomics on the
 // even (odd) positions 2l (2l+1) of a 64-position block hit 32 banks.
 __device__ __forceinline__ int ycol(int j) { return j ^ ((j >> 5) & 1); }
+
+// The two sweeps of an orientation (top-down and bottom-up rows; left-right
+// and right-left columns) add into one fp32 output plane of their own
+// without atomics: before the midpoint each writes only the half of the
+// plane it reaches first (rows / columns below ceil(L/2) for the forward
+// sweep, the rest for the backward one) and stores; after a barrier of the
+// two warps each adds to the half the other stored.  `split` is the first
+// step after the midpoint; with one sweep of the orientation active it
+// stores everywhere.
+__device__ __forceinline__ int sweep_split(bool pair, bool fwd, int L) {
+    return pair ? (fwd ? (L + 1) / 2 : L / 2) : L;
+}
+__device__ __forceinline__ void pair_barrier(int id) {
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+// Branch-free: positions past the end of a line write a dummy column /
+// row of the plane, `first` is warp-uniform.
+__device__ __forceinline__ void put_y(float *a, float v, bool first) {
+    const float o = *a;
+    *a = (first ? 0.0f : o) + v;
+}
 
 // One step of the recurrence: h <- (sum_k P_k h(q+k-1)) / D + lambda x.  The
 // terms that need a neighbour lane's value (from the shuffles) come last.
@@ -268,7 +288,7 @@ __device__ __forceinline__ void recur(float (&h)[R], const LineW<R> &W) {
 // ---------------------------------------------------------------------------
 // Row lines (directions 0 and 1).
 // ---------------------------------------------------------------------------
-template <typename T, int R, bool FWD, int MODE>
+template <typename T, int R, int MODE>
 struct RowScan {
     static constexpr int es = sizeof(T);
     static constexpr int NP = R / 2;            // blocks of position pairs
@@ -287,14 +307,19 @@ struct RowScan {
     int eo[kWords];     // element offset (in a row) of each raw word, clamped into the row
     int cs[R];          // output column of each position in the staged output plane
     const char *gp[kTensors];   // the current item's planes
-    int item_k;                 // index of the current item among this CTA's items
+    // lane t < 6: byte offsets of tensor t's planes of the current and the
+    // next item (-1: none), for the L2 prefetches
+    long long pf_cur, pf_next;
+    const bool fwd;             // top-down (else bottom-up)
+    const int split;            // first step after the midpoint (see sweep_split)
 
     __device__ static int pos(int lane, int r) {
         return r < 2 * NP ? 64 * (r / 2) + 2 * lane + (r & 1) : 64 * NP + lane;
     }
 
     __device__ RowScan(const DirParams &p_, unsigned char *, int lane_, int d)
-        : p(p_), lane(lane_), D(d), L(p_.H), nch(1), total_chunks(0), item_k(0) {
+        : p(p_), lane(lane_), D(d), L(p_.H), nch(1), total_chunks(0), pf_cur(-1), pf_next(-1),
+          fwd(d == 0), split(sweep_split((p_.dirs & 3) == 3, d == 0, p_.H)) {
         const int W = p_.W;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -303,7 +328,8 @@ struct RowScan {
             g.m0[r] = q > 0 ? 1.0f : 0.0f;
             g.m2[r] = q + 1 < W ? 1.0f : 0.0f;
             g.thr[r] = __float_as_int((q > 0 && q + 1 < W) ? 1e11f : 1e5f);
-            cs[r] = q ^ ((q >> 5) & 1);
+            // positions past the row end write the plane's last (dummy) column
+            cs[r] = q < W ? q ^ ((q >> 5) & 1) : p_.y_pitch - 1;
         }
 #pragma unroll
         for (int k = 0; k < kWords; ++k) {
@@ -317,16 +343,25 @@ struct RowScan {
         }
     }
 
-    __device__ __forceinline__ void set_item(int k) {
-        item_k = k;
+    // Byte offset of tensor t's plane of the CTA's k-th item (-1: none).
+    __device__ __forceinline__ long long plane_off(int k, int t) const {
         const int item = blockIdx.x + k * gridDim.x;
+        if (item >= p.n_items) return -1;
         const int plane = item / p.bands;
         const int b = plane / p.Cc, ch = plane - b * p.Cc;
-#pragma unroll
-        for (int t = 0; t < kTensors; ++t) gp[t] = dir_tensor(p, t) + dir_plane(p, b, ch, D, t) * es;
+        return static_cast<long long>(dir_plane(p, b, ch, D, t) * es);
     }
 
-    __device__ __forceinline__ int row_of(int s) const { return FWD ? s : L - 1 - s; }
+    __device__ __forceinline__ void set_item(int k) {
+#pragma unroll
+        for (int t = 0; t < kTensors; ++t) gp[t] = dir_tensor(p, t) + plane_off(k, t);
+        if (lane < kTensors) {
+            pf_cur = plane_off(k, lane);
+            pf_next = plane_off(k + 1, lane);
+        }
+    }
+
+    __device__ __forceinline__ int row_of(int s) const { return fwd ? s : L - 1 - s; }
 
     // Raw words of scan line s (global loads, L2-resident after the prefetch).
     __device__ __forceinline__ void load(int s, Raw &w) const {
@@ -358,45 +393,34 @@ struct RowScan {
     // of the warp's line stream, which continues into its next item.
     __device__ __forceinline__ void prefetch(int s0) const {
         if (lane >= kTensors) return;
-        int k = item_k, s = s0;
-        while (s >= L) { s -= L; ++k; }
-        const int item = blockIdx.x + k * gridDim.x;
-        if (item >= p.n_items) return;
-        const int plane = item / p.bands;
-        const int b = plane / p.Cc, ch = plane - b * p.Cc;
-        const int t = lane;
+        const long long po = s0 < L ? pf_cur : pf_next;
+        const int s = s0 < L ? s0 : s0 - L;
+        if (po < 0 || s >= L) return;
         const int n = min(kPrefetchLines, L - s);
-        const int r0 = FWD ? s : L - s - n;
-        const char *base = dir_tensor(p, t);
-        const unsigned long long end = dir_tensor_bytes(p, t);
-        unsigned long long a = (dir_plane(p, b, ch, D, t) + static_cast<size_t>(r0) * p.W) * es;
+        const int r0 = fwd ? s : L - s - n;
+        const unsigned long long end = dir_tensor_bytes(p, lane);
+        unsigned long long a = static_cast<unsigned long long>(po) + static_cast<unsigned long long>(r0) * p.W * es;
         unsigned long long e = a + static_cast<unsigned long long>(n) * p.W * es;
         a &= ~15ull;
         e = (e + 15) & ~15ull;
         if (e > end) e = end & ~15ull;
-        if (e > a) prefetch_l2(base + a, static_cast<uint32_t>(e - a));
+        if (e > a) prefetch_l2(dir_tensor(p, lane) + a, static_cast<uint32_t>(e - a));
     }
 
-    __device__ __forceinline__ void plain_line(int s, LineW<R> &W) const {
-        Raw w;
-        load(s, w);
-        float v[kTensors][R];
-        unpack(w, v);
-        line_weights_plain_v<R>(v, g, W);
-    }
-
-    // Gated output of the step's row into the output plane / band / global.
-    __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int row, uint32_t ysa,
-                                         float *yg, int band_lo, int band_hi) const {
+    // Gated output of the step's row into the row plane / band / global.
+    __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int row, float *ys,
+                                         float *yg, int band_lo, int band_hi, bool first) const {
         const bool in = MODE != kYBanded || (row >= band_lo && row < band_hi);
-        const uint32_t yl = ysa + 4u * static_cast<uint32_t>((row - band_lo) * p.y_pitch);
+        float *yl = ys + (row - band_lo) * p.y_pitch;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const float cy = W.uu[r] * h[r];
             if (MODE == kYGlobal) {
                 if (g.valid[r]) atomicAdd(yg + static_cast<size_t>(row) * p.W + pos(lane, r), cy);
+            } else if (MODE == kYShared) {
+                if (g.valid[r] && in) atomicAdd(yl + cs[r], cy);
             } else {
-                red_add_shared_if(yl + 4u * cs[r], cy, g.valid[r] && in);
+                if (in) put_y(yl + cs[r], cy, first);
             }
         }
     }
@@ -442,24 +466,23 @@ struct RowScan {
     // Step s (J = s mod 2): the plain form if line s was flagged, the update
     // of line s, the weights of line s+1 (its raw words arrived two steps
     // ago), the loads of line s+3 into the freed buffer, the outputs.
-    template <int J, bool CHECK>
-    __device__ __forceinline__ void step(int s, float (&h)[R], LineW<R> (&Wb)[2], bool (&bad)[2],
-                                         Raw (&rb)[2], uint32_t ysa, float *yg, int band_lo, int band_hi) {
+    template <int J>
+    __device__ __forceinline__ void step(int s, float (&h)[R], LineW<R> (&Wb)[2],
+                                         Raw (&rb)[2], float *ys, float *yg, int band_lo, int band_hi) {
         LineW<R> &Wc = Wb[J];
-        if (__any_sync(0xffffffffu, bad[J])) plain_line(s, Wc);
+        if (MODE != kYGlobal && MODE != kYShared && s == split) pair_barrier(2);
         recur_rows(h, Wc);
-        if (!CHECK || s + 1 < L) {
+        if (s + 1 < L) {
             float v[kTensors][R];
             unpack(rb[J ^ 1], v);
-            bad[J ^ 1] = line_weights(v, g, Wb[J ^ 1]);
-            if (!CHECK || s + 3 < L) load(s + 3, rb[J ^ 1]);
+            line_terms(v, g, Wb[J ^ 1]);
+            if (s + 3 < L) load(s + 3, rb[J ^ 1]);
         }
-        emit(h, Wc, row_of(s), ysa, yg, band_lo, band_hi);
+        emit(h, Wc, row_of(s), ys, yg, band_lo, band_hi, s < split);
     }
 
     // Run every line of the CTA's k-th item.
     __device__ void run_item(int k, float *ys, float *yg, int band_lo, int band_hi) {
-        const uint32_t ysa = smem_u32(ys);
         set_item(k);
         if (k == 0) {
             for (int s0 = 0; s0 < kPrefetchAhead; s0 += kPrefetchLines) prefetch(s0);
@@ -468,29 +491,21 @@ struct RowScan {
 #pragma unroll
         for (int r = 0; r < R; ++r) h[r] = 0.0f;
         LineW<R> Wb[2];
-        bool bad[2];
         Raw rb[2];
         load(0, rb[0]);
         if (L > 1) load(1, rb[1]);
         {
             float v[kTensors][R];
             unpack(rb[0], v);
-            bad[0] = line_weights(v, g, Wb[0]);
+            line_terms(v, g, Wb[0]);
         }
         if (L > 2) load(2, rb[0]);
         int s = 0;
 #pragma unroll 1
-        for (; s + 4 < L; s += 2) {
-            if ((s & (kPrefetchLines - 1)) == 0) prefetch(s + kPrefetchAhead);
-            step<0, false>(s, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
-            step<1, false>(s + 1, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
-        }
-        // the last lines
-#pragma unroll 1
         for (; s < L; s += 2) {
             if ((s & (kPrefetchLines - 1)) == 0) prefetch(s + kPrefetchAhead);
-            step<0, true>(s, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
-            if (s + 1 < L) step<1, true>(s + 1, h, Wb, bad, rb, ysa, yg, band_lo, band_hi);
+            step<0>(s, h, Wb, rb, ys, yg, band_lo, band_hi);
+            if (s + 1 < L) step<1>(s + 1, h, Wb, rb, ys, yg, band_lo, band_hi);
         }
     }
 };
@@ -498,7 +513,7 @@ struct RowScan {
 // ---------------------------------------------------------------------------
 // Column lines (directions 2 and 3).
 // ---------------------------------------------------------------------------
-template <typename T, int R, bool FWD, int MODE>
+template <typename T, int R, int MODE>
 struct ColScan {
     static constexpr int es = sizeof(T);
     static constexpr int NS = kColStages;
@@ -519,9 +534,12 @@ struct ColScan {
     int rowq[R];        // byte offset of strip row q_r in a stage (row 0 when q_r >= H)
     int fsw[R];         // word swizzle of that strip row (see swz)
     bool inb[R];        // q_r is an output row of the current item
-    uint32_t ya[R];     // shared address of column 0 of its output row
+    int yoff[R];        // offset (floats) of its output row in the column plane
     int issue_item;
     const char **gtab;  // [kTensors] planes of the item being issued (shared memory)
+    const bool fwd;     // left-right (else right-left)
+    const int split;    // first step after the midpoint (see sweep_split)
+    const uint32_t selA, selB;   // byte permutations of a bf16 word's columns
 
     __device__ ColScan(const DirParams &p_, unsigned char *smem, int lane_, int d)
         : p(p_), lane(lane_), D(d),
@@ -529,7 +547,11 @@ struct ColScan {
           L(p_.W), nch((p_.W + kColStrip / static_cast<int>(sizeof(T)) - 1) /
                        (kColStrip / static_cast<int>(sizeof(T)))),
           total_chunks(0), issue_item(-1),
-          gtab(reinterpret_cast<const char **>(smem + p_.bar_off + 128 + 64 * (d - 2))) {
+          gtab(reinterpret_cast<const char **>(smem + p_.bar_off + 128 + 64 * (d - 2))),
+          fwd(d == 2), split(sweep_split((p_.dirs & 12) == 12, d == 2, p_.W)),
+          // bf16 word -> float of its first / second column in scan order:
+          // the low half (bits << 16) or the high half (bits & 0xffff0000)
+          selA(d == 2 ? 0x1044u : 0x3244u), selB(d == 2 ? 0x3244u : 0x1044u) {
         g.init(lane_, p_.H);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -547,7 +569,7 @@ struct ColScan {
     __device__ __forceinline__ static int swz(int q) { return es == 2 ? (q / (16 * R)) & 1 : 0; }
 
     // Lowest column of chunk c (chunks are numbered in scan order).
-    __device__ __forceinline__ int chunk_lo(int c) const { return FWD ? c * CH : L - CH - c * CH; }
+    __device__ __forceinline__ int chunk_lo(int c) const { return fwd ? c * CH : L - CH - c * CH; }
 
     __device__ __forceinline__ unsigned char *stage_ptr(int gi) const {
         return ring + (gi % NS) * p.stage_col;
@@ -567,7 +589,7 @@ struct ColScan {
             if (col < 0 || col + 4 / es > L) return;
         }
         // right-to-left scans store the words of a strip row reversed
-        const int dw = FWD ? w : 3 - w;
+        const int dw = fwd ? w : 3 - w;
         const int rowstep = kCopyRows * p.W * es;
         int src_off = (i0 * p.W + lo) * es + 4 * w;
         uint32_t drow = sb + static_cast<uint32_t>(i0 * kColPitch);
@@ -629,7 +651,7 @@ struct ColScan {
 
     // Column K (0 or 1, scan order) of a word set as floats.
     template <int K>
-    __device__ __forceinline__ static void unpack(const PairSet &w, float (&v)[kTensors][R]) {
+    __device__ __forceinline__ void unpack(const PairSet &w, float (&v)[kTensors][R]) const {
 #pragma unroll
         for (int t = 0; t < kTensors; ++t)
 #pragma unroll
@@ -638,8 +660,7 @@ struct ColScan {
                     v[t][r] = __uint_as_float(K == 0 ? w[t][r].x : w[t][r].y);
                 } else {
                     // a word holds columns (2m, 2m+1); reversed sweeps meet the odd one first
-                    const bool hi = FWD ? (K & 1) : !(K & 1);
-                    v[t][r] = __uint_as_float(hi ? (w[t][r] & 0xffff0000u) : (w[t][r] << 16));
+                    v[t][r] = __uint_as_float(prmt0(w[t][r], K == 0 ? selA : selB));
                 }
             }
     }
@@ -647,53 +668,39 @@ struct ColScan {
     // Byte offset, within a strip row's 16-byte piece, of the chunk's step k
     // for position r (swizzled word, then the bf16 half).
     __device__ __forceinline__ int step_byte(int k, int r) const {
-        return es == 4 ? 4 * k : 4 * ((k / 2) ^ fsw[r]) + 2 * (FWD ? (k & 1) : 1 - (k & 1));
+        return es == 4 ? 4 * k : 4 * ((k / 2) ^ fsw[r]) + 2 * (fwd ? (k & 1) : 1 - (k & 1));
     }
 
-    // Step k of the staged chunk gi, read from shared memory.
-    __device__ __forceinline__ void reload(int gi, int k, float (&v)[kTensors][R]) const {
-        const unsigned char *sp = stage_ptr(gi);
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int off = rowq[r] + step_byte(k, r);
-#pragma unroll
-            for (int t = 0; t < kTensors; ++t) v[t][r] = sload<T>(sp + off + 16 * t);
-        }
-    }
-
-    __device__ __forceinline__ void plain(int gi, int k, LineW<R> &W) const {
-        LineAddr<R> a;
-        const unsigned char *sp = stage_ptr(gi);
-#pragma unroll
-        for (int t = 0; t < kTensors; ++t) a.base[t] = sp + 16 * t;
-#pragma unroll
-        for (int r = 0; r < R; ++r) a.off[r] = rowq[r] + step_byte(k, r);
-        line_weights_plain<T, R>(a, g, W);
-    }
-
-    __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int col, float *yg) const {
+    __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int col, float *ys,
+                                         float *yg, bool first) const {
+        const int yc = ycol(col);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const float cy = W.uu[r] * h[r];
             if (MODE == kYGlobal) {
                 if (g.valid[r]) atomicAdd(yg + static_cast<size_t>(lane * R + r) * p.W + col, cy);
+            } else if (MODE == kYShared) {
+                if (inb[r]) atomicAdd(ys + yoff[r] + yc, cy);
             } else {
-                red_add_shared_if(ya[r] + 4u * ycol(col), cy, inb[r]);
+                put_y(ys + yoff[r] + yc, cy, first);
             }
         }
     }
 
-    // Step J of body b of the full chunk c (launch chunk number gi): steps
-    // 0-1 read word set A, steps 2-3 word set B.  B is loaded by step 0; the
-    // next body's A by step 2 (from the next chunk, waited for here, when b
-    // is the chunk's last body); `last` when chunk c ends the item.
+    // Step J of body b of chunk c (launch chunk number gi; n of its CH steps
+    // exist, n < CH only in the item's last chunk): steps 0-1 read word set
+    // A, steps 2-3 word set B.  B is loaded by step 0; the next body's A by
+    // step 2 (from the next chunk, waited for here, when b is the chunk's
+    // last body); `last` when chunk c ends the item.
     template <int J>
-    __device__ __forceinline__ void bstep(int gi, int c, int b, bool last, float (&h)[R],
-                                          LineW<R> (&Wb)[2], bool (&bad)[2], PairSet &A, PairSet &B,
-                                          float *yg) {
+    __device__ __forceinline__ void bstep(int gi, int c, int b, bool last, int n, float (&h)[R],
+                                          LineW<R> (&Wb)[2], PairSet &A, PairSet &B,
+                                          float *ys, float *yg) {
         LineW<R> &Wc = Wb[J & 1];
         const int k = 4 * b + J;   // step within the chunk
-        if (__any_sync(0xffffffffu, bad[J & 1])) plain(gi, k, Wc);
+        if (k >= n) return;
+        const int st = c * CH + k;  // step within the item
+        if (MODE != kYGlobal && MODE != kYShared && st == split) pair_barrier(3);
         recur(h, Wc);
         const bool more = b + 1 < NB || !last;   // a step follows this body's last
         if (J == 0) load_pair(stage_ptr(gi), 2 * b + 1, B);
@@ -706,48 +713,30 @@ struct ColScan {
             }
         }
         // weights of the next step
-        if (J < 3 || more) {
+        if (k + 1 < n || (J == 3 && more)) {
             float v[kTensors][R];
             if (J == 0) unpack<1>(A, v);
             else if (J == 1) unpack<0>(B, v);
             else if (J == 2) unpack<1>(B, v);
             else unpack<0>(A, v);
-            bad[(J + 1) & 1] = line_weights(v, g, Wb[(J + 1) & 1]);
+            line_terms(v, g, Wb[(J + 1) & 1]);
         }
-        emit(h, Wc, FWD ? c * CH + k : L - 1 - c * CH - k, yg);
-    }
-
-    // Step k of the item's last, partial chunk (n < CH steps), reading each
-    // column from shared memory; J = k mod 2 picks the weight set.
-    template <int J>
-    __device__ __forceinline__ void pstep(int gi, int c, int k, int n, float (&h)[R], LineW<R> (&Wb)[2],
-                                          bool (&bad)[2], float *yg) {
-        LineW<R> &Wc = Wb[J];
-        if (__any_sync(0xffffffffu, bad[J])) plain(gi, k, Wc);
-        recur(h, Wc);
-        if (k + 1 < n) {
-            float v[kTensors][R];
-            reload(gi, k + 1, v);
-            bad[J ^ 1] = line_weights(v, g, Wb[J ^ 1]);
-        }
-        emit(h, Wc, FWD ? c * CH + k : L - 1 - c * CH - k, yg);
+        emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
     }
 
     // Run every column of the item whose first chunk is g0.
     __device__ void run_item(int g0, float *ys, float *yg, int band_lo, int band_hi) {
-        const uint32_t ysa = smem_u32(ys);
         float h[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             h[r] = 0.0f;
             const int q = lane * R + r;
             inb[r] = g.valid[r] && (MODE != kYBanded || (q >= band_lo && q < band_hi));
-            ya[r] = ysa + 4u * static_cast<uint32_t>((inb[r] ? q - band_lo : 0) * p.y_pitch);
+            // rows outside the band (or past the end) write the plane's dummy row
+            yoff[r] = (inb[r] ? q - band_lo : p.band_rows) * p.y_pitch;
         }
         LineW<R> Wb[2];
-        bool bad[2];
         PairSet A, B;
-        const int nfull = L / CH;
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
             const int gi = g0 + c;
@@ -757,30 +746,18 @@ struct ColScan {
                 // the item's first chunk: wait for it, weights of step 0
                 wait<1>();
                 float v[kTensors][R];
-                if (nfull > 0) {
-                    load_pair(stage_ptr(gi), 0, A);
-                    unpack<0>(A, v);
-                } else {
-                    reload(gi, 0, v);
-                }
-                bad[0] = line_weights(v, g, Wb[0]);
+                load_pair(stage_ptr(gi), 0, A);
+                unpack<0>(A, v);
+                line_terms(v, g, Wb[0]);
             }
-            if (c < nfull) {
-                const bool last = c + 1 == nch;
+            const bool last = c + 1 == nch;
+            const int n = min(CH, L - c * CH);
 #pragma unroll 1
-                for (int b = 0; b < NB; ++b) {
-                    bstep<0>(gi, c, b, last, h, Wb, bad, A, B, yg);
-                    bstep<1>(gi, c, b, last, h, Wb, bad, A, B, yg);
-                    bstep<2>(gi, c, b, last, h, Wb, bad, A, B, yg);
-                    bstep<3>(gi, c, b, last, h, Wb, bad, A, B, yg);
-                }
-            } else {
-                const int n = L - c * CH;
-#pragma unroll 1
-                for (int k = 0; k < n; k += 2) {
-                    pstep<0>(gi, c, k, n, h, Wb, bad, yg);
-                    if (k + 1 < n) pstep<1>(gi, c, k + 1, n, h, Wb, bad, yg);
-                }
+            for (int b = 0; b < NB; ++b) {
+                bstep<0>(gi, c, b, last, n, h, Wb, A, B, ys, yg);
+                bstep<1>(gi, c, b, last, n, h, Wb, A, B, ys, yg);
+                bstep<2>(gi, c, b, last, n, h, Wb, A, B, ys, yg);
+                bstep<3>(gi, c, b, last, n, h, Wb, A, B, ys, yg);
             }
         }
     }
@@ -794,14 +771,17 @@ __device__ __forceinline__ void dir_barrier() {
 }
 
 // The whole kernel seen from the warp that runs direction D.
-template <typename T, int R, bool ROW, bool FWD, int MODE>
+template <typename T, int R, bool ROW, int MODE>
 __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem, int warp, int lane, int D) {
-    float *ys = reinterpret_cast<float *>(smem);   // output plane or band, fp32 [rows][y_pitch]
+    // output planes (or bands), fp32 [rows][y_pitch]: rows, then columns
+    float *ysr = reinterpret_cast<float *>(smem);
+    float *ysc = reinterpret_cast<float *>(smem + p.ycol_off);
+    const bool has_row = (p.dirs & 3) != 0, has_col = (p.dirs & 12) != 0;
     const int YP = p.y_pitch;
     const bool active = (p.dirs >> D) & 1;
     const int n_my = blockIdx.x < p.n_items ? (p.n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    using Scan = typename std::conditional<ROW, RowScan<T, R, FWD, MODE>, ColScan<T, R, FWD, MODE>>::type;
+    using Scan = typename std::conditional<ROW, RowScan<T, R, MODE>, ColScan<T, R, MODE>>::type;
     Scan sc(p, smem, lane, D);
     const int total = active ? n_my * sc.nch : 0;
     sc.total_chunks = total;
@@ -822,19 +802,27 @@ __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem
             for (int e = threadIdx.x; e < p.H * p.W; e += kDirThreads) yg[e] = 0.0f;
             dir_barrier();
         }
-        if (active) sc.run_item(ROW ? k : k * sc.nch, ys, yg, band_lo, band_hi);
+        if (active) sc.run_item(ROW ? k : k * sc.nch, (ROW || MODE == kYShared) ? ysr : ysc, yg, band_lo, band_hi);
         dir_barrier();
         if (MODE != kYGlobal) {
-            // write the band out once (converted) and clear it for the next item
+            // the sum of the two planes, written out once (converted); every
+            // position of a plane is stored again by the next item
             T *outp = static_cast<T *>(p.out) + static_cast<size_t>(plane) * p.H * p.W +
                       static_cast<size_t>(band_lo) * p.W;
             for (int i = warp; i < band_hi - band_lo; i += 4) {
-                float *yr = ys + i * YP;
+                float *yr = ysr + i * YP;
+                const float *yc = ysc + i * YP;
                 T *orow = outp + static_cast<size_t>(i) * p.W;
                 for (int j = lane; j < p.W; j += 32) {
-                    const int yc = ycol(j);
-                    orow[j] = from_f<T>(yr[yc]);
-                    yr[yc] = 0.0f;
+                    const int c = ycol(j);
+                    if (MODE == kYShared) {
+                        // the single plane is accumulated into: clear it
+                        orow[j] = from_f<T>(yr[c]);
+                        yr[c] = 0.0f;
+                    } else {
+                        const float v = (has_row ? yr[c] : 0.0f) + (has_col ? yc[c] : 0.0f);
+                        orow[j] = from_f<T>(v);
+                    }
                 }
             }
             dir_barrier();
@@ -857,12 +845,10 @@ prop2d_dir_kernel(const DirParams p) {
         for (int e = threadIdx.x; e < p.bar_off / 16; e += kDirThreads) z[e] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    switch (warp) {
-        case 0: dir_role<T, R, true, true, MODE>(p, smem, warp, lane, 0); break;
-        case 1: dir_role<T, R, true, false, MODE>(p, smem, warp, lane, 1); break;
-        case 2: dir_role<T, R, false, true, MODE>(p, smem, warp, lane, 2); break;
-        default: dir_role<T, R, false, false, MODE>(p, smem, warp, lane, 3); break;
-    }
+    // the two sweeps of an orientation share one code path (the sweep sign
+    // is a runtime value), which halves the instruction footprint
+    if (warp < 2) dir_role<T, R, true, MODE>(p, smem, warp, lane, warp);
+    else dir_role<T, R, false, MODE>(p, smem, warp, lane, warp);
 }
 
 }  // namespace gspn
