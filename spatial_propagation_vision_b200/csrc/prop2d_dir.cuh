@@ -130,7 +130,7 @@ __device__ __forceinline__ unsigned long long dir_tensor_bytes(const DirParams &
 // Per-line normalisation terms and gates of the lane's R positions.
 template <int R>
 struct LineW {
-    float P0[R], P1[R], P2[R], rD[R], bx[R], uu[R];
+    float w0[R], w1[R], w2[R], bx[R], uu[R];   // w_k: normalised weight of slot k
 };
 
 // Per-lane constants of a line of M positions.
@@ -178,11 +178,12 @@ __device__ __forceinline__ bool line_weights(const float (&v)[kTensors][R], cons
         const float2 P2 = __fmul2_rn(__fmul2_rn(a0, a1), mm2);
         const float2 Dn = __fadd2_rn(__fadd2_rn(P0, P1), P2);
         bad |= (__float_as_int(Dn.x) > g.thr[r]) | (__float_as_int(Dn.y) > g.thr[r + 1]);
+        const float2 rD = make_float2(rcp(Dn.x), rcp(Dn.y));
+        const float2 w0 = __fmul2_rn(P0, rD), w1 = __fmul2_rn(P1, rD), w2 = __fmul2_rn(P2, rD);
         const float2 bx = __fmul2_rn(make_float2(v[0][r], v[0][r + 1]), make_float2(v[5][r], v[5][r + 1]));
-        W.P0[r] = P0.x; W.P0[r + 1] = P0.y;
-        W.P1[r] = P1.x; W.P1[r + 1] = P1.y;
-        W.P2[r] = P2.x; W.P2[r + 1] = P2.y;
-        W.rD[r] = rcp(Dn.x); W.rD[r + 1] = rcp(Dn.y);
+        W.w0[r] = w0.x; W.w0[r + 1] = w0.y;
+        W.w1[r] = w1.x; W.w1[r + 1] = w1.y;
+        W.w2[r] = w2.x; W.w2[r + 1] = w2.y;
         W.bx[r] = bx.x; W.bx[r + 1] = bx.y;
         W.uu[r] = v[1][r]; W.uu[r + 1] = v[1][r + 1];
     }
@@ -196,10 +197,10 @@ __device__ __forceinline__ bool line_weights(const float (&v)[kTensors][R], cons
         const float P2 = a0 * a1 * g.m2[r];
         const float Dn = (P0 + P1) + P2;
         bad |= __float_as_int(Dn) > g.thr[r];
-        W.P0[r] = P0;
-        W.P1[r] = P1;
-        W.P2[r] = P2;
-        W.rD[r] = rcp(Dn);
+        const float rD = rcp(Dn);
+        W.w0[r] = P0 * rD;
+        W.w1[r] = P1 * rD;
+        W.w2[r] = P2 * rD;
         W.bx[r] = v[0][r] * v[5][r];
         W.uu[r] = v[1][r];
     }
@@ -207,7 +208,7 @@ __device__ __forceinline__ bool line_weights(const float (&v)[kTensors][R], cons
 }
 
 // Plain-form terms of one line (rare path): the normalised weights go in
-// P0..P2 with rD = 1, so the update is the same for both forms.  Same
+// w0..w2 like the fast form's.  Same
 // arithmetic as the fast form's exponentials and reciprocals, without
 // products: sigmoid(z) = 1 / (1 + 2^(-z log2 e)) saturates to 0 or 1 instead
 // of overflowing, and the clamp of the local sum is explicit.
@@ -221,10 +222,9 @@ __device__ __forceinline__ void line_weights_plain_v(const float (&v)[kTensors][
         const float s1 = rcp(1.0f + ex2(v[3][r] * nl2e));
         const float s2 = rcp(1.0f + ex2(v[4][r] * nl2e)) * g.m2[r];
         const float iS = rcp(fmaxf((s0 + s1) + s2, 1e-6f));
-        W.P0[r] = s0 * iS;
-        W.P1[r] = s1 * iS;
-        W.P2[r] = s2 * iS;
-        W.rD[r] = 1.0f;
+        W.w0[r] = s0 * iS;
+        W.w1[r] = s1 * iS;
+        W.w2[r] = s2 * iS;
         W.bx[r] = v[0][r] * v[5][r];
         W.uu[r] = v[1][r];
     }
@@ -236,6 +236,13 @@ __device__ __forceinline__ void line_weights_plain_v(const float (&v)[kTensors][
 template <int R>
 __device__ __forceinline__ void line_terms(const float (&v)[kTensors][R], const LaneGeom<R> &g, LineW<R> &W) {
     const bool bad = line_weights(v, g, W);
+    if (__any_sync(0xffffffffu, bad)) line_weights_plain_v<R>(v, g, W);
+}
+// The same check as a separate call, so that a step can place it (a branch,
+// which ends a straight-line block) after the rest of its work.
+template <int R>
+__device__ __forceinline__ void line_terms_fix(bool bad, const float (&v)[kTensors][R], const LaneGeom<R> &g,
+                                               LineW<R> &W) {
     if (__any_sync(0xffffffffu, bad)) line_weights_plain_v<R>(v, g, W);
 }
 
@@ -251,9 +258,9 @@ __device__ __forceinline__ int ycol(int j) { return j ^ ((j >> 5) & 1); }
 // sweep, the rest for the backward one) and stores; after a barrier of the
 // two warps each adds to the half the other stored.  `split` is the first
 // step after the midpoint; with one sweep of the orientation active it
-// stores everywhere.
+// stores everywhere (split = L + 1: no barrier).
 __device__ __forceinline__ int sweep_split(bool pair, bool fwd, int L) {
-    return pair ? (fwd ? (L + 1) / 2 : L / 2) : L;
+    return pair ? (fwd ? (L + 1) / 2 : L / 2) : L + 1;
 }
 __device__ __forceinline__ void pair_barrier(int id) {
     asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
@@ -274,12 +281,12 @@ __device__ __forceinline__ void recur(float (&h)[R], const LineW<R> &W) {
     float hn[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        float N = W.P1[r] * h[r];
-        if (r > 0) N = fmaf(W.P0[r], h[r - 1], N);
-        if (r < R - 1) N = fmaf(W.P2[r], h[r + 1], N);
-        if (r == 0) N = fmaf(W.P0[r], hl, N);
-        if (r == R - 1) N = fmaf(W.P2[r], hr, N);
-        hn[r] = fmaf(N, W.rD[r], W.bx[r]);
+        float N = fmaf(W.w1[r], h[r], W.bx[r]);
+        if (r > 0) N = fmaf(W.w0[r], h[r - 1], N);
+        if (r < R - 1) N = fmaf(W.w2[r], h[r + 1], N);
+        if (r == 0) N = fmaf(W.w0[r], hl, N);
+        if (r == R - 1) N = fmaf(W.w2[r], hr, N);
+        hn[r] = N;
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) h[r] = hn[r];
@@ -454,10 +461,9 @@ struct RowScan {
         float hn[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            float N = W.P1[r] * h[r];
-            N = fmaf(W.P0[r], left[r], N);
-            N = fmaf(W.P2[r], right[r], N);
-            hn[r] = fmaf(N, W.rD[r], W.bx[r]);
+            float N = fmaf(W.w1[r], h[r], W.bx[r]);
+            N = fmaf(W.w0[r], left[r], N);
+            hn[r] = fmaf(W.w2[r], right[r], N);
         }
 #pragma unroll
         for (int r = 0; r < R; ++r) h[r] = hn[r];
@@ -470,15 +476,16 @@ struct RowScan {
     __device__ __forceinline__ void step(int s, float (&h)[R], LineW<R> (&Wb)[2],
                                          Raw (&rb)[2], float *ys, float *yg, int band_lo, int band_hi) {
         LineW<R> &Wc = Wb[J];
-        if (MODE != kYGlobal && MODE != kYShared && s == split) pair_barrier(2);
         recur_rows(h, Wc);
-        if (s + 1 < L) {
-            float v[kTensors][R];
-            unpack(rb[J ^ 1], v);
-            line_terms(v, g, Wb[J ^ 1]);
-            if (s + 3 < L) load(s + 3, rb[J ^ 1]);
-        }
+        // weights of line s+1 (past the last line: stale but finite words,
+        // never used) and the loads of line s+3 (clamped into the plane)
+        float v[kTensors][R];
+        unpack(rb[J ^ 1], v);
+        const bool bad = line_weights(v, g, Wb[J ^ 1]);
+        load(min(s + 3, L - 1), rb[J ^ 1]);
         emit(h, Wc, row_of(s), ys, yg, band_lo, band_hi, s < split);
+        line_terms_fix(bad, v, g, Wb[J ^ 1]);
+        if (MODE != kYGlobal && MODE != kYShared && s + 1 == split) pair_barrier(2);
     }
 
     // Run every line of the CTA's k-th item.
@@ -493,13 +500,13 @@ struct RowScan {
         LineW<R> Wb[2];
         Raw rb[2];
         load(0, rb[0]);
-        if (L > 1) load(1, rb[1]);
+        load(min(1, L - 1), rb[1]);
         {
             float v[kTensors][R];
             unpack(rb[0], v);
             line_terms(v, g, Wb[0]);
         }
-        if (L > 2) load(2, rb[0]);
+        load(min(2, L - 1), rb[0]);
         int s = 0;
 #pragma unroll 1
         for (; s < L; s += 2) {
@@ -700,7 +707,6 @@ struct ColScan {
         const int k = 4 * b + J;   // step within the chunk
         if (k >= n) return;
         const int st = c * CH + k;  // step within the item
-        if (MODE != kYGlobal && MODE != kYShared && st == split) pair_barrier(3);
         recur(h, Wc);
         const bool more = b + 1 < NB || !last;   // a step follows this body's last
         if (J == 0) load_pair(stage_ptr(gi), 2 * b + 1, B);
@@ -712,16 +718,17 @@ struct ColScan {
                 load_pair(stage_ptr(gi + 1), 0, A);
             }
         }
-        // weights of the next step
-        if (k + 1 < n || (J == 3 && more)) {
-            float v[kTensors][R];
-            if (J == 0) unpack<1>(A, v);
-            else if (J == 1) unpack<0>(B, v);
-            else if (J == 2) unpack<1>(B, v);
-            else unpack<0>(A, v);
-            line_terms(v, g, Wb[(J + 1) & 1]);
-        }
+        // weights of the next step (when none follows: stale but finite
+        // words, never used)
+        float v[kTensors][R];
+        if (J == 0) unpack<1>(A, v);
+        else if (J == 1) unpack<0>(B, v);
+        else if (J == 2) unpack<1>(B, v);
+        else unpack<0>(A, v);
+        const bool bad = line_weights(v, g, Wb[(J + 1) & 1]);
         emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
+        line_terms_fix(bad, v, g, Wb[(J + 1) & 1]);
+        if (MODE != kYGlobal && MODE != kYShared && st + 1 == split) pair_barrier(3);
     }
 
     // Run every column of the item whose first chunk is g0.
