@@ -186,7 +186,7 @@ def cpu_inputs_f64(w, seed=0, planes=None):
     return {k: v.double().numpy() for k, v in inp.items()}
 
 
-def cpu_oracle_baseline(w, budget_s=12.0, max_passes=3):
+def cpu_oracle_baseline(w, budget_s=12.0, max_passes=20):
     """The oracle as it stands, one host core, on whole passes over the
     workload's planes (repeated until about budget_s)."""
     inp = cpu_inputs_f64(w)
