@@ -303,8 +303,13 @@ struct RowScan {
     // raw words of one line per tensor: bf16 pairs share a 32-bit word
     static constexpr int kWords = es == 2 ? NP + (kSingle ? 1 : 0) : R;
     using Raw = uint32_t[kTensors][kWords];
+    // Raw words of the next kDepth lines are in flight in registers; the loop
+    // body is kUnroll steps so that both the two weight sets and the kDepth
+    // raw buffers are indexed statically.
+    static constexpr int kDepth = 3;
+    static constexpr int kUnroll = kDepth % 2 == 0 ? kDepth : 2 * kDepth;
     static constexpr int kPrefetchAhead = 16;   // lines between an L2 prefetch and its use
-    static constexpr int kPrefetchLines = 8;    // lines per prefetch
+    static constexpr int kPrefetchLines = kUnroll;   // lines per prefetch (one per loop body)
 
     const DirParams &p;
     const int lane, D;
@@ -474,18 +479,31 @@ struct RowScan {
     // ago), the loads of line s+3 into the freed buffer, the outputs.
     template <int J>
     __device__ __forceinline__ void step(int s, float (&h)[R], LineW<R> (&Wb)[2],
-                                         Raw (&rb)[2], float *ys, float *yg, int band_lo, int band_hi) {
-        LineW<R> &Wc = Wb[J];
+                                         Raw (&rb)[kDepth], float *ys, float *yg, int band_lo, int band_hi) {
+        constexpr int cur = J & 1, nxt = (J + 1) & 1, buf = (J + 1) % kDepth;
+        LineW<R> &Wc = Wb[cur];
         recur_rows(h, Wc);
         // weights of line s+1 (past the last line: stale but finite words,
-        // never used) and the loads of line s+3 (clamped into the plane)
+        // never used) and the loads of line s+1+kDepth into the freed buffer
+        // (clamped into the plane)
         float v[kTensors][R];
-        unpack(rb[J ^ 1], v);
-        const bool bad = line_weights(v, g, Wb[J ^ 1]);
-        load(min(s + 3, L - 1), rb[J ^ 1]);
+        unpack(rb[buf], v);
+        const bool bad = line_weights(v, g, Wb[nxt]);
+        load(min(s + 1 + kDepth, L - 1), rb[buf]);
         emit(h, Wc, row_of(s), ys, yg, band_lo, band_hi, s < split);
-        line_terms_fix(bad, v, g, Wb[J ^ 1]);
+        line_terms_fix(bad, v, g, Wb[nxt]);
         if (MODE != kYGlobal && MODE != kYShared && s + 1 == split) pair_barrier(2);
+    }
+
+    template <int J>
+    __device__ __forceinline__ void steps(int s, float (&h)[R], LineW<R> (&Wb)[2], Raw (&rb)[kDepth],
+                                          float *ys, float *yg, int band_lo, int band_hi) {
+        if constexpr (J < kUnroll) {
+            if (J == 0 || s + J < L) {
+                step<J>(s + J, h, Wb, rb, ys, yg, band_lo, band_hi);
+                steps<J + 1>(s, h, Wb, rb, ys, yg, band_lo, band_hi);
+            }
+        }
     }
 
     // Run every line of the CTA's k-th item.
@@ -498,21 +516,19 @@ struct RowScan {
 #pragma unroll
         for (int r = 0; r < R; ++r) h[r] = 0.0f;
         LineW<R> Wb[2];
-        Raw rb[2];
-        load(0, rb[0]);
-        load(min(1, L - 1), rb[1]);
+        Raw rb[kDepth];
+#pragma unroll
+        for (int m = 0; m < kDepth; ++m) load(min(m, L - 1), rb[m]);
         {
             float v[kTensors][R];
             unpack(rb[0], v);
             line_terms(v, g, Wb[0]);
         }
-        load(min(2, L - 1), rb[0]);
-        int s = 0;
+        load(min(kDepth, L - 1), rb[0]);
 #pragma unroll 1
-        for (; s < L; s += 2) {
-            if ((s & (kPrefetchLines - 1)) == 0) prefetch(s + kPrefetchAhead);
-            step<0>(s, h, Wb, rb, ys, yg, band_lo, band_hi);
-            if (s + 1 < L) step<1>(s + 1, h, Wb, rb, ys, yg, band_lo, band_hi);
+        for (int s = 0; s < L; s += kUnroll) {
+            prefetch(s + kPrefetchAhead);
+            steps<0>(s, h, Wb, rb, ys, yg, band_lo, band_hi);
         }
     }
 };
