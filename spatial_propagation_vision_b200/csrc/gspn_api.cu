@@ -176,12 +176,13 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
         const int caps[4] = {dp.smem_per_sm / 4 - 1024, dp.smem_per_sm / 3 - 1024,
                              dp.smem_per_sm / 2 - 1024, dp.smem_optin};
         bool fit = false;
-        // two planes; then one plane with shared atomics (bf16) or global
-        // atomics (fp32); then bands
-        const int order[4] = {0, 3, 1, 2};
-        for (int oi = 0; oi < 4 && !fit; ++oi) {
-            const int mode = order[oi];
-            if ((mode == 1 && es != 4) || (mode == 3 && es != 2)) continue;
+        // bf16: one plane with shared atomics (the four directions run
+        // uncoupled until the end of an item), else bands; fp32: two planes
+        // (atomic-free), one plane, global atomics, else bands
+        const int order_bf16[2] = {3, 2}, order_f32[4] = {0, 3, 1, 2};
+        const int n_order = es == 2 ? 2 : 4;
+        for (int oi = 0; oi < n_order && !fit; ++oi) {
+            const int mode = es == 2 ? order_bf16[oi] : order_f32[oi];
             for (int ci = 0; ci < 4 && !fit; ++ci) {
                 const int cap = caps[ci] < dp.smem_optin ? caps[ci] : dp.smem_optin;
                 fit = plan_dir_fit(pl, cap, H, W, dirs, mode);
@@ -197,12 +198,12 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
             const bool banded = pl.p.bands > 1;
             if (es == 4) {
                 err = pl.y_global ? launch_dir_f32_global(R, pl, dp, stream, g_last)
+                      : pl.y_shared ? launch_dir_f32_shared(R, pl, dp, stream, g_last)
                       : banded    ? launch_dir_f32_banded(R, pl, dp, stream, g_last)
                                   : launch_dir_f32_smem(R, pl, dp, stream, g_last);
             } else {
                 err = pl.y_shared ? launch_dir_bf16_shared(R, pl, dp, stream, g_last)
-                      : banded    ? launch_dir_bf16_banded(R, pl, dp, stream, g_last)
-                                  : launch_dir_bf16_smem(R, pl, dp, stream, g_last);
+                                  : launch_dir_bf16_banded(R, pl, dp, stream, g_last);
             }
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }

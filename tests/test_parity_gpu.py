@@ -173,10 +173,12 @@ def test_extreme_logits(gspn, mode, dtype):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "dir"),
+    ((2, 3, 74, 74), "bf16", "dir-shared"),
+    ((2, 3, 74, 74), "f32", "dir"),
+    ((1, 2, 160, 160), "f32", "dir-shared"),   # two output planes do not fit
     ((1, 2, 256, 256), "f32", "dir-yglobal"),
     ((1, 2, 256, 256), "bf16", "dir-banded"),
-    ((1, 2, 148, 148), "bf16", "dir-shared"),   # two output planes do not fit
+    ((1, 2, 148, 148), "bf16", "dir-shared"),
     ((1, 2, 20, 33), "bf16", "generic"),       # odd bf16 row width
     ((1, 1, 300, 40), "f32", "generic"),       # line longer than 256
     ((2, 2, 1, 40), "bf16", "generic"),        # lines of one position
