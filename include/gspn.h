@@ -18,8 +18,11 @@
  * on-grid neighbours, a clamp of that sum at 1e-6 and a divide (Sec. 5.1
  * "Fused CUDA normalization"; papernotes.org normalisation formula).  Slot k
  * names the absolute orthogonal offset k-1 (-1 = left for row lines, up for
- * column lines); off-grid slots carry no weight.  The normalisation is fused
- * into the scan: the weights are never written anywhere.
+ * column lines); off-grid slots carry no weight.  With per-channel logits
+ * the normalisation is fused into the scan and the weights are never
+ * written anywhere.  In the compact mode (share_w = 1, one logit field shared
+ * by all channels), gspn_prop2d_fwd_ws normalises each shared field once
+ * into a caller-provided workspace and every channel's scan reads it.
  *
  * Layouts (element offsets, contiguous, row-major):
  *   x      [B][Cc][H][W]
@@ -32,10 +35,11 @@
  * slots not enabled by `dirs` are never read.
  *
  * Dtypes: inputs and output share one dtype (fp32 or bf16); the recurrence
- * state, the weights and the direction sum are fp32.
+ * state, the weight arithmetic and the direction sum are fp32 (the bf16
+ * compact mode's workspace stores its normalised weights as fp16).
  *
- * Ownership: the caller owns every buffer.  The library keeps no state
- * between calls and allocates no memory.
+ * Ownership: the caller owns every buffer, the workspace included.  The
+ * library keeps no state between calls and allocates no memory.
  *
  * Errors: every entry point returns a gspn_status and never aborts or traps.
  * Argument errors are detected on the host before anything is launched;
@@ -64,7 +68,8 @@ typedef enum {
     GSPN_ERR_DTYPE = 4,    /* unknown gspn_dtype */
     GSPN_ERR_ALIGN = 5,    /* a device pointer is not 16-byte aligned */
     GSPN_ERR_CUDA = 6,     /* the CUDA runtime reported an error */
-    GSPN_ERR_DEVICE = 7    /* the current device is not sm_100 (B200) */
+    GSPN_ERR_DEVICE = 7,   /* the current device is not sm_100 (B200) */
+    GSPN_ERR_WORKSPACE = 8 /* workspace smaller than gspn_prop2d_workspace_bytes */
 } gspn_status;
 
 enum {
@@ -99,6 +104,43 @@ gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const void *wlogi
                             const void *u, int B, int Cc, int H, int W, int dirs,
                             int share_w, gspn_dtype dtype, void *out,
                             cudaStream_t stream);
+
+/*
+ * gspn_prop2d_workspace_bytes -- size of the workspace gspn_prop2d_fwd_ws
+ * needs for these arguments: B*4*3*H*W elements (fp32 for GSPN_F32, fp16 for
+ * GSPN_BF16) when share_w = 1, else 0.  Returns 0 for invalid arguments.
+ */
+size_t gspn_prop2d_workspace_bytes(int B, int Cc, int H, int W, int dirs, int share_w,
+                                   gspn_dtype dtype);
+
+/*
+ * gspn_prop2d_fwd_ws -- gspn_prop2d_fwd with a workspace for the compact mode
+ * (Sec. 4.2 "Channel-shared weights": one weight field per position, shared
+ * across channels).
+ *
+ * With share_w = 1, a first kernel normalises the shared logits of every
+ * (batch, enabled direction, position) once into `workspace`, layout
+ * [B][4][3][H][W]: slot 0 = w0, slot 1 = w0 + w1 + w2 (1 unless the clamp
+ * binds), slot 2 = w2, in fp32 (GSPN_F32) or fp16 (GSPN_BF16); the scans of
+ * all Cc channels then read those weights instead of normalising per
+ * channel.  fp16 weights carry a relative rounding error of at most 2^-11
+ * each; w1 is formed as the difference, so a position's weights keep their
+ * exact sum.  With share_w = 0 the workspace is not used (may be NULL) and
+ * the call equals gspn_prop2d_fwd.
+ *
+ * workspace      : device pointer, 16-byte aligned, at least
+ *                  gspn_prop2d_workspace_bytes(...) bytes; overwritten; must
+ *                  not alias any other argument.  Stream-ordered: it may be
+ *                  reused by the next call on the same stream.
+ * workspace_size : its size in bytes.
+ * Other arguments and errors as gspn_prop2d_fwd, plus GSPN_ERR_NULL for a
+ * NULL workspace and GSPN_ERR_WORKSPACE for one that is too small (share_w = 1).
+ * gspn_last_launch_info then counts two launches.
+ */
+gspn_status gspn_prop2d_fwd_ws(const void *x, const void *lambda, const void *wlogit,
+                               const void *u, int B, int Cc, int H, int W, int dirs,
+                               int share_w, gspn_dtype dtype, void *out, void *workspace,
+                               size_t workspace_size, cudaStream_t stream);
 
 /*
  * gspn_prop2d_fwd_host -- the same operation on HOST buffers.

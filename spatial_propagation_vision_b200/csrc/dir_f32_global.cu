@@ -1,10 +1,11 @@
-// Direction kernel variant: element type float, output mode kYGlobal.
+// Direction kernel variant: element type float, output mode kYGlobal,
+// weights normalised in the scan.
 #include "dir_launch.cuh"
 
 namespace gspn_host {
 
 cudaError_t launch_dir_f32_global(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li) {
-    return launch_dir_r<float, gspn::kYGlobal>(R, pl, dp, s, li);
+    return launch_dir_r<float, gspn::kYGlobal, false>(R, pl, dp, s, li);
 }
 
 }  // namespace gspn_host

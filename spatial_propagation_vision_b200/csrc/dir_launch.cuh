@@ -6,9 +6,9 @@
 
 namespace gspn_host {
 
-template <typename T, int R, int MODE>
+template <typename T, int R, int MODE, bool PRE>
 cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t stream, LaunchInfo &li) {
-    auto kern = gspn::prop2d_dir_kernel<T, R, MODE>;
+    auto kern = gspn::prop2d_dir_kernel<T, R, MODE, PRE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -29,17 +29,17 @@ cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t 
     return cudaGetLastError();
 }
 
-template <typename T, int MODE>
+template <typename T, int MODE, bool PRE>
 cudaError_t launch_dir_r(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li) {
     switch (R) {
-        case 1: return launch_dir_t<T, 1, MODE>(pl, dp, s, li);
-        case 2: return launch_dir_t<T, 2, MODE>(pl, dp, s, li);
-        case 3: return launch_dir_t<T, 3, MODE>(pl, dp, s, li);
-        case 4: return launch_dir_t<T, 4, MODE>(pl, dp, s, li);
-        case 5: return launch_dir_t<T, 5, MODE>(pl, dp, s, li);
-        case 6: return launch_dir_t<T, 6, MODE>(pl, dp, s, li);
-        case 7: return launch_dir_t<T, 7, MODE>(pl, dp, s, li);
-        case 8: return launch_dir_t<T, 8, MODE>(pl, dp, s, li);
+        case 1: return launch_dir_t<T, 1, MODE, PRE>(pl, dp, s, li);
+        case 2: return launch_dir_t<T, 2, MODE, PRE>(pl, dp, s, li);
+        case 3: return launch_dir_t<T, 3, MODE, PRE>(pl, dp, s, li);
+        case 4: return launch_dir_t<T, 4, MODE, PRE>(pl, dp, s, li);
+        case 5: return launch_dir_t<T, 5, MODE, PRE>(pl, dp, s, li);
+        case 6: return launch_dir_t<T, 6, MODE, PRE>(pl, dp, s, li);
+        case 7: return launch_dir_t<T, 7, MODE, PRE>(pl, dp, s, li);
+        case 8: return launch_dir_t<T, 8, MODE, PRE>(pl, dp, s, li);
         default: return cudaErrorInvalidValue;
     }
 }

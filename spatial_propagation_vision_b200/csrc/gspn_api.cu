@@ -122,6 +122,7 @@ extern "C" const char *gspn_status_str(gspn_status s) {
         case GSPN_ERR_NULL: return "GSPN_ERR_NULL: a required pointer is NULL";
         case GSPN_ERR_SHAPE: return "GSPN_ERR_SHAPE: unsupported or negative size";
         case GSPN_ERR_DIRS: return "GSPN_ERR_DIRS: dirs must be 1..15 and share_w 0 or 1";
+        case GSPN_ERR_WORKSPACE: return "GSPN_ERR_WORKSPACE: workspace smaller than gspn_prop2d_workspace_bytes";
         case GSPN_ERR_DTYPE: return "GSPN_ERR_DTYPE: unknown dtype";
         case GSPN_ERR_ALIGN: return "GSPN_ERR_ALIGN: device pointers must be 16-byte aligned";
         case GSPN_ERR_CUDA: return "GSPN_ERR_CUDA: CUDA runtime error";
@@ -139,10 +140,37 @@ extern "C" void gspn_last_launch_info(int *launches, int *grid, int *block, int 
     if (path) *path = g_last.path;
 }
 
-extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const void *wlogit,
-                                       const void *u, int B, int Cc, int H, int W, int dirs,
-                                       int share_w, gspn_dtype dtype, void *out,
-                                       cudaStream_t stream) {
+namespace {
+
+// Bytes of the compact mode's normalised weights: [B][4][1][3][H][W] of fp32
+// (fp32 inputs) or fp16 (bf16 inputs).
+size_t workspace_bytes(int B, int H, int W, int share_w, gspn_dtype dtype) {
+    if (!share_w || B <= 0 || H <= 0 || W <= 0) return 0;
+    const size_t es = dtype == GSPN_BF16 ? 2 : 4;
+    return static_cast<size_t>(B) * 4 * 3 * H * W * es;
+}
+
+using DirLaunch = cudaError_t (*)(int, const DirPlan &, const DeviceProps &, cudaStream_t, LaunchInfo &);
+
+// The direction kernel variant for (element size, output path, weights
+// normalised ahead).
+DirLaunch dir_variant(int es, const DirPlan &pl, bool pre) {
+    const bool banded = pl.p.bands > 1;
+    if (es == 4) {
+        if (pl.y_global) return pre ? launch_dir_f32_global_pre : launch_dir_f32_global;
+        if (pl.y_shared) return pre ? launch_dir_f32_shared_pre : launch_dir_f32_shared;
+        if (banded) return pre ? launch_dir_f32_banded_pre : launch_dir_f32_banded;
+        return pre ? launch_dir_f32_smem_pre : launch_dir_f32_smem;
+    }
+    if (pl.y_shared) return pre ? launch_dir_bf16_shared_pre : launch_dir_bf16_shared;
+    return pre ? launch_dir_bf16_banded_pre : launch_dir_bf16_banded;
+}
+
+// gspn_prop2d_fwd with an optional workspace (compact mode only: the
+// weights are then normalised once into it and read by every channel).
+gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
+                       int Cc, int H, int W, int dirs, int share_w, gspn_dtype dtype, void *out,
+                       void *ws, cudaStream_t stream) {
     g_last = LaunchInfo{};
     if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
     if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
@@ -195,16 +223,15 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
             pl.p.end_gate = 4ULL * pl.p.end_x;
             pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane_bytes;
             if (status_word(&pl.p.status) != cudaSuccess) return GSPN_ERR_CUDA;
-            const bool banded = pl.p.bands > 1;
-            if (es == 4) {
-                err = pl.y_global ? launch_dir_f32_global(R, pl, dp, stream, g_last)
-                      : pl.y_shared ? launch_dir_f32_shared(R, pl, dp, stream, g_last)
-                      : banded    ? launch_dir_f32_banded(R, pl, dp, stream, g_last)
-                                  : launch_dir_f32_smem(R, pl, dp, stream, g_last);
-            } else {
-                err = pl.y_shared ? launch_dir_bf16_shared(R, pl, dp, stream, g_last)
-                                  : launch_dir_bf16_banded(R, pl, dp, stream, g_last);
+            const bool pre = share_w && ws;
+            if (pre) {
+                // the compact mode's weights, normalised once for all channels
+                gspn::NormParams np{wlogit, ws, B, H, W, dirs};
+                if (launch_norm(np, es == 2, dp, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+                pl.p.wl = ws;
             }
+            err = dir_variant(es, pl, pre)(R, pl, dp, stream, g_last);
+            if (pre) g_last.launches += 1;
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }
     }
@@ -215,6 +242,40 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
     err = launch_generic(gp, es == 2, dp, stream, fits, g_last);
     if (!fits) return GSPN_ERR_SHAPE;
     return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const void *wlogit,
+                                       const void *u, int B, int Cc, int H, int W, int dirs,
+                                       int share_w, gspn_dtype dtype, void *out,
+                                       cudaStream_t stream) {
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, share_w, dtype, out, nullptr, stream);
+}
+
+extern "C" size_t gspn_prop2d_workspace_bytes(int B, int Cc, int H, int W, int dirs, int share_w,
+                                              gspn_dtype dtype) {
+    if (Cc < 0 || dirs < 1 || dirs > 15 || (dtype != GSPN_F32 && dtype != GSPN_BF16)) return 0;
+    return workspace_bytes(B, H, W, share_w, dtype);
+}
+
+extern "C" gspn_status gspn_prop2d_fwd_ws(const void *x, const void *lambda, const void *wlogit,
+                                          const void *u, int B, int Cc, int H, int W, int dirs,
+                                          int share_w, gspn_dtype dtype, void *out, void *workspace,
+                                          size_t workspace_size, cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
+    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
+    if (dtype != GSPN_F32 && dtype != GSPN_BF16) return GSPN_ERR_DTYPE;
+    if (B == 0 || Cc == 0 || H == 0 || W == 0) return GSPN_OK;
+    const size_t need = workspace_bytes(B, H, W, share_w, dtype);
+    if (need > 0) {
+        if (!workspace) return GSPN_ERR_NULL;
+        if (workspace_size < need) return GSPN_ERR_WORKSPACE;
+        if (misaligned(workspace)) return GSPN_ERR_ALIGN;
+    }
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, share_w, dtype, out,
+                      need > 0 ? workspace : nullptr, stream);
 }
 
 extern "C" gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda,

@@ -9,6 +9,7 @@
 
 #include "prop2d_dir.cuh"
 #include "prop2d_generic.cuh"
+#include "prop2d_norm.cuh"
 
 namespace gspn_host {
 
@@ -32,14 +33,23 @@ struct DirPlan {
 
 inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
-// Direction kernel, one function per (element type, output mode); R is the
-// positions per lane (1..8).
+// Direction kernel, one function per (element type, output mode, weights
+// normalised in the scan or ahead: _pre); R is the positions per lane (1..8).
 cudaError_t launch_dir_f32_smem(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_f32_smem_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_banded(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_f32_banded_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_global(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_f32_global_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_shared(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_f32_shared_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_banded(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_banded_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_shared(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_shared_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+
+// Normalised weights of the compact mode into the workspace (one launch).
+cudaError_t launch_norm(const gspn::NormParams &np, bool bf16, const DeviceProps &dp, cudaStream_t s);
 
 // General kernel; `fits` is false when even one output row does not fit.
 cudaError_t launch_generic(const gspn::GenericParams &gp, bool bf16, const DeviceProps &dp,

@@ -3,54 +3,59 @@
 // One CTA of four warps owns one (batch, channel) plane (or one band of its
 // output rows when the fp32 output plane does not fit in shared memory);
 // warp d runs direction d: 0 top->bottom, 1 bottom->top (row lines),
-// 2 left->right, 3 right->left (column lines).  Lane l holds the R
-// consecutive positions q = l*R + r of the current line in registers; the
-// neighbours across lanes come from shuffles.  Each warp runs code compiled
-// for its own direction (orientation and sweep sign are template
-// parameters), so the line and offset arithmetic inside a chunk is static.
+// 2 left->right, 3 right->left (column lines).  The two sweeps of an
+// orientation share one code path with a runtime sweep sign, which halves
+// the instruction footprint.  Lane l holds R positions of the current line
+// in registers: for row lines positions 2l and 2l+1 of every 64-position
+// block (one 32-bit word of bf16) plus 64*(R/2) + l when R is odd; for
+// column lines the R consecutive positions q = l*R + r.  Neighbours held by
+// another lane come from shuffles.
 //
 // Normalisation (Sec. 5.1 "Fused CUDA normalization": sigmoid, local sum,
 // clamp, divide), folded into the update.  With a_k = 1 + exp(-z_k),
 // sigmoid(z_k) = 1 / a_k and, for P_k = product of a_j over the other
-// on-grid slots j != k and D = sum_k P_k,
-//     h = sum_k w_k h_prev(q+k-1) + lambda x = (sum_k P_k h_prev(q+k-1)) / D + lambda x,
-// which takes three exponentials and one reciprocal per position.  An
-// off-grid slot takes a_k = 1, P_k = 0.  Whenever the clamp of the
-// denominator could bind, or a product overflows, D exceeds a threshold
-// (1e11 with three on-grid slots, 1e5 with two) or is not finite; the
-// weights of that line are then recomputed in the plain form.  The weights
-// of line s+1 do not depend on the hidden state; they are computed in the
-// same straight block as line s's update, and the weight sets of
-// consecutive lines alternate between two register sets.
+// on-grid slots j != k and D = sum_k P_k, w_k = P_k / D: three exponentials
+// and one reciprocal per position.  An off-grid slot takes a_k = 1, P_k = 0.
+// Whenever the clamp of the denominator could bind, or a product overflows,
+// D exceeds a threshold (1e11 with three on-grid slots, 1e5 with two) or is
+// not finite; the weights of that line are then recomputed in the plain
+// form.  The weights of line s+1 do not depend on the hidden state; they are
+// computed in the same block as line s's update, alternating between two
+// register sets.  In the compact mode with a workspace (PRE), the weights
+// were normalised ahead once for all channels (prop2d_norm.cuh) and are read.
 //
-// Input staging in shared memory:
-//   * row lines: a chunk of t_row rows is one contiguous span per tensor;
-//     lane t < 6 moves tensor t's span with one bulk copy (TMA engine) into
-//     a 16-byte aligned slot of a three-stage ring and arrives on the
-//     stage's mbarrier; the lanes then read their positions of a line with
-//     16-bit loads;
+// Input staging:
+//   * row lines: each lane loads its words of a line straight from global
+//     memory (read-only path), three lines ahead into registers; one lane
+//     per tensor issues a bulk L2 prefetch (TMA engine) of the lines about
+//     to be read, eight lines ahead, continuing into the warp's next plane;
 //   * column lines: a chunk is a strip of 16 bytes of every grid row (8 bf16
-//     or 4 fp32 columns).  The strip rows of the six tensors are interleaved
-//     (104-byte pitch: six 16-byte pieces and 8 bytes of padding, so that
-//     the lanes' 8-byte reads hit distinct banks).  Each lane copies
-//     (4-byte cp.async) and later reads its own R rows, so it waits for its
-//     own copies only.  One 8-byte read per tensor and position brings half
-//     a strip (4 bf16 / 2 fp32 columns) into registers.  Right-to-left
-//     scans store the words of a strip row in reverse order, so both sweeps
-//     meet their columns in scan order.
-// The gated outputs u * h of the four directions are summed into one fp32
-// plane in shared memory with shared-memory atomics and written once.
+//     or 4 fp32 columns), copied by the warp with 4-byte cp.async (four lanes
+//     per grid row) into a two-stage ring.  The strip rows of the six tensors
+//     are interleaved (104-byte pitch); bf16 words are XOR-swizzled on
+//     alternate bands of 16R rows so the lanes' reads hit 32 banks, and
+//     right-to-left sweeps store the words of a strip row in reverse order,
+//     so both sweeps meet their columns in scan order.  A four-step body
+//     reads two-column words.
+// Outputs u * h are accumulated in fp32 in shared memory and written once,
+// converted, at the end of the plane (modes below): one plane that all
+// directions add into with shared-memory atomics, or two planes (rows,
+// columns) written without atomics, each shared by a sweep pair that splits
+// at the midpoint; global atomics and row bands cover planes too large for
+// shared memory.
 //
 // Positions past the end of a line (q >= M) compute finite garbage that
 // never reaches a valid position: their right-hand neighbour term of
 // position M-1 has P_2 = 0.  For that they read finite values only: the
 // rings are zeroed at launch and afterwards hold copies of the inputs
-// (column lanes past the end read grid row 0's strip).
+// (column lanes past the end read grid row 0's strip; row lanes read a
+// clamped in-plane word).
 #pragma once
 
 #include <cstdint>
 #include <type_traits>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "device_common.cuh"
 
@@ -246,6 +251,48 @@ __device__ __forceinline__ void line_terms_fix(bool bad, const float (&v)[kTenso
     if (__any_sync(0xffffffffu, bad)) line_weights_plain_v<R>(v, g, W);
 }
 
+// Terms of one line whose weights were normalised ahead of the scan (the
+// compact mode's weights, shared by every channel): slots 2, 3 and 4 hold w0,
+// the sum of the three weights and w2, so w1 is their difference and the
+// weights of a position sum exactly to that sum (1 unless the clamp bound).
+template <int R>
+__device__ __forceinline__ void line_pre(const float (&v)[kTensors][R], LineW<R> &W) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        W.w0[r] = v[2][r];
+        W.w2[r] = v[4][r];
+        W.w1[r] = (v[3][r] - v[2][r]) - v[4][r];
+        W.bx[r] = v[0][r] * v[5][r];
+        W.uu[r] = v[1][r];
+    }
+}
+
+// Weights of the next line from its unpacked inputs: computed from the
+// logits (fast form, flagged lines redone in the plain form by
+// line_terms_fix), or read when they were normalised ahead (PRE).
+template <bool PRE, int R>
+__device__ __forceinline__ bool next_weights(const float (&v)[kTensors][R], const LaneGeom<R> &g, LineW<R> &W) {
+    if constexpr (PRE) {
+        line_pre(v, W);
+        return false;
+    } else {
+        return line_weights(v, g, W);
+    }
+}
+template <bool PRE, int R>
+__device__ __forceinline__ void first_weights(const float (&v)[kTensors][R], const LaneGeom<R> &g, LineW<R> &W) {
+    if constexpr (PRE) line_pre(v, W);
+    else line_terms(v, g, W);
+}
+
+// 16-bit half `hi` of a word as an fp32 value: bf16 bits, or (a weight
+// normalised ahead, for bf16 inputs) fp16.
+template <bool F16>
+__device__ __forceinline__ float half_word(uint32_t w, bool hi) {
+    if constexpr (F16) return __half2float(__ushort_as_half(static_cast<unsigned short>(hi ? (w >> 16) : w)));
+    else return __uint_as_float(hi ? (w & 0xffff0000u) : (w << 16));
+}
+
 // Column of output position j in a staged output row: bit 0 of j is flipped
 // in every other 32-column block, so that the row lanes' atomics on the
 // even (odd) positions 2l (2l+1) of a 64-position block hit 32 banks.
@@ -295,7 +342,7 @@ __device__ __forceinline__ void recur(float (&h)[R], const LineW<R> &W) {
 // ---------------------------------------------------------------------------
 // Row lines (directions 0 and 1).
 // ---------------------------------------------------------------------------
-template <typename T, int R, int MODE>
+template <typename T, int R, int MODE, bool PRE>
 struct RowScan {
     static constexpr int es = sizeof(T);
     static constexpr int NP = R / 2;            // blocks of position pairs
@@ -308,7 +355,7 @@ struct RowScan {
     // raw buffers are indexed statically.
     static constexpr int kDepth = 3;
     static constexpr int kUnroll = kDepth % 2 == 0 ? kDepth : 2 * kDepth;
-    static constexpr int kPrefetchAhead = 16;   // lines between an L2 prefetch and its use
+    static constexpr int kPrefetchAhead = 8;    // lines between an L2 prefetch and its use
     static constexpr int kPrefetchLines = kUnroll;   // lines per prefetch (one per loop body)
 
     const DirParams &p;
@@ -390,14 +437,19 @@ struct RowScan {
         }
     }
 
+    // (weights normalised ahead are fp16 when the inputs are bf16)
     __device__ __forceinline__ static void unpack(const Raw &w, float (&v)[kTensors][R]) {
 #pragma unroll
         for (int t = 0; t < kTensors; ++t)
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                if (es == 4) v[t][r] = __uint_as_float(w[t][r]);
-                else if (r < 2 * NP) v[t][r] = __uint_as_float((r & 1) ? (w[t][r / 2] & 0xffff0000u) : (w[t][r / 2] << 16));
-                else v[t][r] = __uint_as_float(w[t][NP] << 16);
+                if constexpr (es == 4) {
+                    v[t][r] = __uint_as_float(w[t][r]);
+                } else {
+                    const uint32_t word = r < 2 * NP ? w[t][r / 2] : w[t][NP];
+                    const bool hi = r < 2 * NP && (r & 1);
+                    v[t][r] = (PRE && t >= 2 && t <= 4) ? half_word<true>(word, hi) : half_word<false>(word, hi);
+                }
             }
     }
 
@@ -488,10 +540,10 @@ struct RowScan {
         // (clamped into the plane)
         float v[kTensors][R];
         unpack(rb[buf], v);
-        const bool bad = line_weights(v, g, Wb[nxt]);
+        const bool bad = next_weights<PRE>(v, g, Wb[nxt]);
         load(min(s + 1 + kDepth, L - 1), rb[buf]);
         emit(h, Wc, row_of(s), ys, yg, band_lo, band_hi, s < split);
-        line_terms_fix(bad, v, g, Wb[nxt]);
+        if (!PRE) line_terms_fix(bad, v, g, Wb[nxt]);
         if (MODE != kYGlobal && MODE != kYShared && s + 1 == split) pair_barrier(2);
     }
 
@@ -522,7 +574,7 @@ struct RowScan {
         {
             float v[kTensors][R];
             unpack(rb[0], v);
-            line_terms(v, g, Wb[0]);
+            first_weights<PRE>(v, g, Wb[0]);
         }
         load(min(kDepth, L - 1), rb[0]);
 #pragma unroll 1
@@ -536,7 +588,7 @@ struct RowScan {
 // ---------------------------------------------------------------------------
 // Column lines (directions 2 and 3).
 // ---------------------------------------------------------------------------
-template <typename T, int R, int MODE>
+template <typename T, int R, int MODE, bool PRE>
 struct ColScan {
     static constexpr int es = sizeof(T);
     static constexpr int NS = kColStages;
@@ -681,6 +733,9 @@ struct ColScan {
             for (int r = 0; r < R; ++r) {
                 if constexpr (es == 4) {
                     v[t][r] = __uint_as_float(K == 0 ? w[t][r].x : w[t][r].y);
+                } else if (PRE && t >= 2 && t <= 4) {
+                    // fp16 weight normalised ahead: the half met K-th in scan order
+                    v[t][r] = half_word<true>(w[t][r], (K == 0) != fwd);
                 } else {
                     // a word holds columns (2m, 2m+1); reversed sweeps meet the odd one first
                     v[t][r] = __uint_as_float(prmt0(w[t][r], K == 0 ? selA : selB));
@@ -741,9 +796,9 @@ struct ColScan {
         else if (J == 1) unpack<0>(B, v);
         else if (J == 2) unpack<1>(B, v);
         else unpack<0>(A, v);
-        const bool bad = line_weights(v, g, Wb[(J + 1) & 1]);
+        const bool bad = next_weights<PRE>(v, g, Wb[(J + 1) & 1]);
         emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
-        line_terms_fix(bad, v, g, Wb[(J + 1) & 1]);
+        if (!PRE) line_terms_fix(bad, v, g, Wb[(J + 1) & 1]);
         if (MODE != kYGlobal && MODE != kYShared && st + 1 == split) pair_barrier(3);
     }
 
@@ -771,7 +826,7 @@ struct ColScan {
                 float v[kTensors][R];
                 load_pair(stage_ptr(gi), 0, A);
                 unpack<0>(A, v);
-                line_terms(v, g, Wb[0]);
+                first_weights<PRE>(v, g, Wb[0]);
             }
             const bool last = c + 1 == nch;
             const int n = min(CH, L - c * CH);
@@ -794,7 +849,7 @@ __device__ __forceinline__ void dir_barrier() {
 }
 
 // The whole kernel seen from the warp that runs direction D.
-template <typename T, int R, bool ROW, int MODE>
+template <typename T, int R, bool ROW, int MODE, bool PRE>
 __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem, int warp, int lane, int D) {
     // output planes (or bands), fp32 [rows][y_pitch]: rows, then columns
     float *ysr = reinterpret_cast<float *>(smem);
@@ -804,7 +859,7 @@ __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem
     const bool active = (p.dirs >> D) & 1;
     const int n_my = blockIdx.x < p.n_items ? (p.n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    using Scan = typename std::conditional<ROW, RowScan<T, R, MODE>, ColScan<T, R, MODE>>::type;
+    using Scan = typename std::conditional<ROW, RowScan<T, R, MODE, PRE>, ColScan<T, R, MODE, PRE>>::type;
     Scan sc(p, smem, lane, D);
     const int total = active ? n_my * sc.nch : 0;
     sc.total_chunks = total;
@@ -856,7 +911,7 @@ __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem
 
 // Lines of up to 96 positions keep three CTAs (12 warps) per SM: the
 // register budget is then 168 per thread.
-template <typename T, int R, int MODE>
+template <typename T, int R, int MODE, bool PRE>
 __global__ void __launch_bounds__(kDirThreads, R <= 3 ? 3 : 2)
 prop2d_dir_kernel(const DirParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
@@ -870,8 +925,8 @@ prop2d_dir_kernel(const DirParams p) {
     __syncthreads();
     // the two sweeps of an orientation share one code path (the sweep sign
     // is a runtime value), which halves the instruction footprint
-    if (warp < 2) dir_role<T, R, true, MODE>(p, smem, warp, lane, warp);
-    else dir_role<T, R, false, MODE>(p, smem, warp, lane, warp);
+    if (warp < 2) dir_role<T, R, true, MODE, PRE>(p, smem, warp, lane, warp);
+    else dir_role<T, R, false, MODE, PRE>(p, smem, warp, lane, warp);
 }
 
 }  // namespace gspn

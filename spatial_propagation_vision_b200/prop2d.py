@@ -24,11 +24,17 @@ lib = ctypes.CDLL(LIB_PATH)
 
 GSPN_F32, GSPN_BF16 = 0, 1
 STATUS = {0: "GSPN_OK", 1: "GSPN_ERR_NULL", 2: "GSPN_ERR_SHAPE", 3: "GSPN_ERR_DIRS",
-          4: "GSPN_ERR_DTYPE", 5: "GSPN_ERR_ALIGN", 6: "GSPN_ERR_CUDA", 7: "GSPN_ERR_DEVICE"}
+          4: "GSPN_ERR_DTYPE", 5: "GSPN_ERR_ALIGN", 6: "GSPN_ERR_CUDA", 7: "GSPN_ERR_DEVICE",
+          8: "GSPN_ERR_WORKSPACE"}
 
 _vp, _i = ctypes.c_void_p, ctypes.c_int
 lib.gspn_prop2d_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
 lib.gspn_prop2d_fwd.restype = _i
+lib.gspn_prop2d_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                   ctypes.c_size_t, _vp]
+lib.gspn_prop2d_fwd_ws.restype = _i
+lib.gspn_prop2d_workspace_bytes.argtypes = [_i] * 7
+lib.gspn_prop2d_workspace_bytes.restype = ctypes.c_size_t
 lib.gspn_prop2d_fwd_host.argtypes = [_vp] * 10 + [_i] * 7 + [_vp]
 lib.gspn_prop2d_fwd_host.restype = _i
 lib.gspn_status_str.argtypes = [_i]
@@ -69,15 +75,25 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream)
 
 
+def workspace_bytes(B: int, Cc: int, H: int, W: int, dirs: int = 15, share_w: int = 0,
+                    dtype: torch.dtype = torch.float32) -> int:
+    """Bytes of workspace gspn_prop2d_fwd_ws uses (0 unless share_w)."""
+    return int(lib.gspn_prop2d_workspace_bytes(B, Cc, H, W, int(dirs), int(share_w), _DT[dtype]))
+
+
 def prop2d_fwd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torch.Tensor,
                dirs: int = 15, share_w: int = 0, out: torch.Tensor | None = None,
-               stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+               stream: torch.cuda.Stream | None = None,
+               workspace: torch.Tensor | None = None) -> torch.Tensor:
     """y = Prop2D(x; u, lambda, w) on the GPU (gspn_prop2d_fwd).
 
     x [B,Cc,H,W]; lam, u [B,4,Cc,H,W]; wlogit [B,4,Cw,3,H,W] (Cw = 1 if share_w
     else Cc); all float32 or all bfloat16, contiguous, on one CUDA device.
     Returns ``out`` ([B,Cc,H,W], same dtype), allocated if not given.
-    Asynchronous on ``stream`` (default: the current stream).
+    Asynchronous on ``stream`` (default: the current stream).  With
+    ``workspace`` (a contiguous CUDA tensor of at least ``workspace_bytes``
+    bytes) the call goes through gspn_prop2d_fwd_ws: in the compact mode the
+    shared weights are then normalised once for all channels.
     """
     B, Cc, H, W = _dims(x)
     if x.dtype not in _DT:
@@ -94,9 +110,18 @@ def prop2d_fwd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torc
         out = torch.empty((B, Cc, H, W), dtype=x.dtype, device=dev)
     _check("out", out, (B, Cc, H, W), x.dtype, dev)
     with torch.cuda.device(dev):
-        st = lib.gspn_prop2d_fwd(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(), u.data_ptr(),
-                                 B, Cc, H, W, int(dirs), int(share_w), _DT[x.dtype],
-                                 out.data_ptr(), _stream_handle(stream))
+        if workspace is None:
+            st = lib.gspn_prop2d_fwd(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(), u.data_ptr(),
+                                     B, Cc, H, W, int(dirs), int(share_w), _DT[x.dtype],
+                                     out.data_ptr(), _stream_handle(stream))
+        else:
+            if not workspace.is_contiguous() or workspace.device != dev:
+                raise ValueError(f"workspace must be a contiguous tensor on {dev}")
+            st = lib.gspn_prop2d_fwd_ws(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(),
+                                        u.data_ptr(), B, Cc, H, W, int(dirs), int(share_w),
+                                        _DT[x.dtype], out.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream_handle(stream))
     if st != 0:
         raise GspnError(st)
     return out

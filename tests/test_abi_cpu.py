@@ -71,6 +71,46 @@ def test_argument_checks(lib, args, status):
 def test_status_strings(lib):
     lib.gspn_status_str.argtypes = [ctypes.c_int]
     lib.gspn_status_str.restype = ctypes.c_char_p
-    for s in range(8):
+    for s in range(9):
         assert lib.gspn_status_str(s).decode().startswith("GSPN_")
     assert lib.gspn_status_str(99) is not None
+
+
+def _fwd_ws(lib):
+    f = lib.gspn_prop2d_fwd_ws
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 7 + [ctypes.c_void_p] * 2 + \
+                 [ctypes.c_size_t, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    return f
+
+
+def test_workspace_bytes(lib):
+    f = lib.gspn_prop2d_workspace_bytes
+    f.argtypes = [ctypes.c_int] * 7
+    f.restype = ctypes.c_size_t
+    # [B][4][3][H][W] fp32 (fp32 inputs) or fp16 (bf16 inputs), compact mode only
+    assert f(8, 64, 148, 148, 15, 1, 1) == 8 * 4 * 3 * 148 * 148 * 2
+    assert f(2, 3, 5, 7, 15, 1, 0) == 2 * 4 * 3 * 5 * 7 * 4
+    assert f(8, 64, 148, 148, 15, 0, 1) == 0      # per-channel logits: none
+    assert f(8, 64, 148, 148, 0, 1, 1) == 0       # invalid mask
+    assert f(8, 64, 148, 148, 15, 1, 9) == 0      # invalid dtype
+    assert f(0, 64, 148, 148, 15, 1, 1) == 0      # empty
+
+
+N = 2 * 4 * 3 * 8 * 8 * 4   # workspace bytes of B=2, 8x8, fp32
+
+
+@pytest.mark.parametrize("ws,size,status", [
+    (None, N, 1),          # compact mode without a workspace
+    (P, N - 4, 8),         # too small
+    (P + 8, N, 5),         # misaligned
+])
+def test_workspace_checks(lib, ws, size, status):
+    assert _fwd_ws(lib)(P, P, P, P, 2, 4, 8, 8, 15, 1, 0, P, ws, size, None) == status
+
+
+def test_workspace_ignored_without_share_w(lib):
+    # per-channel logits: the workspace is not looked at, the other checks still apply
+    assert _fwd_ws(lib)(None, P, P, P, 2, 4, 8, 8, 15, 0, 0, P, None, 0, None) == 1
+    assert _fwd_ws(lib)(P, P, P, P, 2, 4, 8, 8, 16, 0, 0, P, None, 0, None) == 3
+    assert _fwd_ws(lib)(None, None, None, None, 0, 4, 8, 8, 15, 1, 0, None, None, 0, None) == 0

@@ -46,9 +46,16 @@ def oracle_planes(inp, planes, dirs, share_w):
     return np.stack(out)
 
 
-def check(gspn, inp, dirs=15, share_w=0, planes=None, what=""):
+def workspace(gspn, inp, dirs=15, share_w=1):
+    B, Cc, H, W = inp["x"].shape
+    n = gspn.workspace_bytes(B, Cc, H, W, dirs, share_w, inp["x"].dtype)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+
+
+def check(gspn, inp, dirs=15, share_w=0, planes=None, what="", ws=False):
     d = to_dev(inp)
-    y = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=dirs, share_w=share_w)
+    kw = {"workspace": workspace(gspn, inp, dirs, share_w)} if ws else {}
+    y = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=dirs, share_w=share_w, **kw)
     torch.cuda.synchronize()
     yg = f64(y)
     if planes is None:
@@ -122,6 +129,70 @@ def test_share_w(gspn, shape, dtype):
     B, Cc, H, W = shape
     inp = make_inputs(B, Cc, H, W, share_w=1, sigma_w=1.0, dtype=dtype, seed=7)
     check(gspn, inp, share_w=1, what=f"share_w {shape}")
+
+
+# --------------------------------------------------------------------------
+# compact mode with a workspace: the shared weights normalised once
+# --------------------------------------------------------------------------
+
+def test_workload_2k_workspace(gspn):
+    """The 2k compact workload through gspn_prop2d_fwd_ws (sampled planes)."""
+    w = WORKLOADS["2k"]
+    inp = workload_inputs(w, seed=0)
+    rng = np.random.default_rng(1)
+    planes = [(0, 0), (w.B - 1, w.Cc - 1)] + [(int(rng.integers(w.B)), int(rng.integers(w.Cc)))
+                                              for _ in range(8)]
+    check(gspn, inp, share_w=1, planes=planes, what="2k ws", ws=True)
+    assert gspn.launch_info()["launches"] == 2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1), (2, 5, 16, 16), (3, 4, 37, 38), (2, 3, 74, 74),
+                                   (1, 3, 148, 148), (1, 2, 31, 97), (1, 2, 256, 256),
+                                   (1, 2, 2, 40), (1, 3, 17, 1)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_share_w_workspace(gspn, shape, dtype):
+    B, Cc, H, W = shape
+    inp = make_inputs(B, Cc, H, W, share_w=1, sigma_w=2.0, dtype=dtype, seed=17)
+    check(gspn, inp, share_w=1, what=f"share_w ws {shape} {dtype}", ws=True)
+
+
+@pytest.mark.parametrize("dirs", [1, 2, 4, 8, 5, 10, 15])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_share_w_workspace_masks(gspn, dirs, dtype):
+    inp = make_inputs(2, 3, 21, 18, share_w=1, sigma_w=2.0, dtype=dtype, seed=dirs)
+    check(gspn, inp, dirs=dirs, share_w=1, what=f"ws dirs={dirs}", ws=True)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["clamp_binds", "all_very_negative", "saturated_positive"])
+def test_share_w_workspace_extremes(gspn, mode, dtype):
+    """The clamp (sum of the weights below 1) and saturated logits through the
+    weights normalised ahead."""
+    inp = make_inputs(2, 3, 19, 23, share_w=1, sigma_w=1.0, dtype="f32", seed=3)
+    g = torch.Generator().manual_seed(6)
+    shape = inp["wlogit"].shape
+    if mode == "clamp_binds":
+        wl = -16.0 - 4.0 * torch.rand(shape, generator=g)
+    elif mode == "all_very_negative":
+        wl = -40.0 - 20.0 * torch.rand(shape, generator=g)
+    else:
+        wl = 30.0 + 60.0 * torch.rand(shape, generator=g)
+    inp["wlogit"] = wl
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    inp = {k: v.to(td) for k, v in inp.items()}
+    check(gspn, inp, share_w=1, what=f"ws {mode} {dtype}", ws=True)
+
+
+def test_workspace_unused_without_share_w(gspn):
+    inp = make_inputs(2, 3, 30, 30, sigma_w=2.0, dtype="bf16", seed=2)
+    d = to_dev(inp)
+    y0 = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"])
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    y1 = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], workspace=ws)
+    torch.cuda.synchronize()
+    assert gspn.launch_info()["launches"] == 1
+    assert torch.equal(y0, y1)
 
 
 # --------------------------------------------------------------------------
