@@ -2,7 +2,8 @@
 
 A step is one gspn_prop2d_fwd call over one batch of the workload (default:
 the C-GSPN 1K layer, B=32, Cc=64, 74x74, bf16 inputs, fp32 state, four
-directions, per-channel weights), inputs resident in HBM.  The metric is
+directions, per-channel weights), inputs resident in HBM; compact-mode
+workloads (shared weights) call gspn_prop2d_fwd_ws with a workspace.  The metric is
 Prop2D forward GB/s of algorithmic traffic (x once; lambda, u and the three
 logits once per direction; y once), whole job over all ranks.
 
@@ -278,9 +279,17 @@ def run_ours(args, w):
     if nbytes <= L2_BYTES:
         flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
+    # the compact mode normalises its shared weights once per call into a
+    # workspace allocated here, outside the timed region
+    kw = {}
+    if w.share_w:
+        B, Cc, H, W = d["x"].shape
+        nws = prop2d.workspace_bytes(B, Cc, H, W, w.dirs, w.share_w, d["x"].dtype)
+        kw["workspace"] = torch.empty(nws, dtype=torch.uint8, device=dev)
+
     def call():
         prop2d.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=w.dirs,
-                          share_w=w.share_w, out=out, stream=stream)
+                          share_w=w.share_w, out=out, stream=stream, **kw)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):

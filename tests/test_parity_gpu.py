@@ -79,7 +79,8 @@ def check(gspn, inp, dirs=15, share_w=0, planes=None, what="", ws=False):
 @pytest.mark.parametrize("name", ["tiny", "mid"])
 def test_workload_full(gspn, name):
     w = WORKLOADS[name]
-    check(gspn, workload_inputs(w, seed=0), share_w=w.share_w, what=name)
+    rel = check(gspn, workload_inputs(w, seed=0), share_w=w.share_w, what=name)
+    print(f"\n{name}: max|err| / max|y| = {rel:.3e}")
 
 
 @pytest.mark.parametrize("name", ["1k", "2k", "orig"])
@@ -92,7 +93,8 @@ def test_workload_sampled_planes(gspn, name):
     n = 3 if name == "orig" else 8
     planes = [(0, 0), (w.B - 1, w.Cc - 1)]
     planes += [(int(rng.integers(w.B)), int(rng.integers(w.Cc))) for _ in range(n)]
-    check(gspn, inp, share_w=w.share_w, planes=planes, what=name)
+    rel = check(gspn, inp, share_w=w.share_w, planes=planes, what=name)
+    print(f"\n{name} (sampled planes): max|err| / max|y| = {rel:.3e}")
 
 
 # --------------------------------------------------------------------------
@@ -142,7 +144,8 @@ def test_workload_2k_workspace(gspn):
     rng = np.random.default_rng(1)
     planes = [(0, 0), (w.B - 1, w.Cc - 1)] + [(int(rng.integers(w.B)), int(rng.integers(w.Cc)))
                                               for _ in range(8)]
-    check(gspn, inp, share_w=1, planes=planes, what="2k ws", ws=True)
+    rel = check(gspn, inp, share_w=1, planes=planes, what="2k ws", ws=True)
+    print(f"\n2k with workspace (sampled planes): max|err| / max|y| = {rel:.3e}")
     assert gspn.launch_info()["launches"] == 2
 
 
