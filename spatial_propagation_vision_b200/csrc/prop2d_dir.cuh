@@ -32,11 +32,10 @@
 //   * column lines: a chunk is a strip of 16 bytes of every grid row (8 bf16
 //     or 4 fp32 columns), copied by the warp with 4-byte cp.async (four lanes
 //     per grid row) into a two-stage ring.  The strip rows of the six tensors
-//     are interleaved (104-byte pitch); bf16 words are XOR-swizzled on
-//     alternate bands of 16R rows so the lanes' reads hit 32 banks, and
-//     right-to-left sweeps store the words of a strip row in reverse order,
-//     so both sweeps meet their columns in scan order.  A four-step body
-//     reads two-column words.
+//     are interleaved (104-byte pitch), and right-to-left sweeps store the
+//     words of a strip row in reverse order, so both sweeps meet their
+//     columns in scan order.  A four-step body reads its columns with one
+//     8-byte read per tensor and position (bf16; two for fp32).
 // Outputs u * h are accumulated in fp32 in shared memory and written once,
 // converted, at the end of the plane (modes below): one plane that all
 // directions add into with shared-memory atomics, or two planes (rows,
@@ -352,8 +351,10 @@ struct RowScan {
     using Raw = uint32_t[kTensors][kWords];
     // Raw words of the next kDepth lines are in flight in registers; the loop
     // body is kUnroll steps so that both the two weight sets and the kDepth
-    // raw buffers are indexed statically.
-    static constexpr int kDepth = 3;
+    // raw buffers are indexed statically.  Three lines while a line's words
+    // fit 18 registers, fewer for longer lines so that the lookahead stays
+    // within about 54 registers (beyond that the kernel spills).
+    static constexpr int kDepth = kTensors * kWords <= 18 ? 3 : kTensors * kWords <= 24 ? 2 : 1;
     static constexpr int kUnroll = kDepth % 2 == 0 ? kDepth : 2 * kDepth;
     static constexpr int kPrefetchAhead = 8;    // lines between an L2 prefetch and its use
     static constexpr int kPrefetchLines = kUnroll;   // lines per prefetch (one per loop body)
@@ -607,7 +608,6 @@ struct ColScan {
     int total_chunks;
     LaneGeom<R> g;
     int rowq[R];        // byte offset of strip row q_r in a stage (row 0 when q_r >= H)
-    int fsw[R];         // word swizzle of that strip row (see swz)
     bool inb[R];        // q_r is an output row of the current item
     int yoff[R];        // offset (floats) of its output row in the column plane
     int issue_item;
@@ -632,16 +632,13 @@ struct ColScan {
         for (int r = 0; r < R; ++r) {
             const int q = lane_ * R + r < p_.H ? lane_ * R + r : 0;
             rowq[r] = q * kColPitch;
-            fsw[r] = swz(q);
         }
     }
 
-    // bf16 strips are read one 32-bit word per lane (all 32 lanes in one
-    // wavefront): lanes l and l+16 read rows 48 apart (R = 3), whose 104-byte
-    // pitches put them on the same bank, so bit 0 of the word index within a
-    // strip row is flipped on every other band of 16R rows.  fp32 strips are
-    // read 64 bits per lane, half a warp per wavefront, already conflict-free.
-    __device__ __forceinline__ static int swz(int q) { return es == 2 ? (q / (16 * R)) & 1 : 0; }
+    // bf16 strips are read 64 bits per lane (a body's four columns of a
+    // tensor): lanes l < 16 read rows 3l + r, whose 104-byte pitches put
+    // each half-warp's 8-byte reads on distinct bank pairs; fp32 strips are
+    // read 64 bits per lane too (two columns).
 
     // Lowest column of chunk c (chunks are numbered in scan order).
     __device__ __forceinline__ int chunk_lo(int c) const { return fwd ? c * CH : L - CH - c * CH; }
@@ -670,7 +667,7 @@ struct ColScan {
         uint32_t drow = sb + static_cast<uint32_t>(i0 * kColPitch);
 #pragma unroll 1
         for (int row = i0; row < p.H; row += kCopyRows) {
-            const uint32_t dst = drow + 4u * static_cast<uint32_t>(dw ^ swz(row));
+            const uint32_t dst = drow + 4u * static_cast<uint32_t>(dw);
 #pragma unroll
             for (int t = 0; t < kTensors; ++t) cp_async_4(dst + 16 * t, gt[t] + src_off);
             src_off += rowstep;
@@ -710,17 +707,32 @@ struct ColScan {
         __syncwarp();
     }
 
-    // Word set of the column pair `pidx` (0..3 in scan order within a strip
-    // row; always even or always odd at a given call site) of a stage.
+    // fp32: word set of the column pair `pidx` (0..3 in scan order within a
+    // strip row) of a stage, 8 bytes per tensor and position.
     __device__ __forceinline__ void load_pair(const unsigned char *sp, int pidx, PairSet &w) const {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            // word (pidx ^ fsw) of the bf16 strip row; fp32 pairs are 8 bytes
-            const int off = es == 2 ? rowq[r] + 4 * pidx + ((pidx & 1) ? -4 : 4) * fsw[r]
-                                    : rowq[r] + 8 * pidx;
+            const int off = rowq[r] + 8 * pidx;
 #pragma unroll
             for (int t = 0; t < kTensors; ++t)
                 w[t][r] = *reinterpret_cast<const Pair *>(sp + off + 16 * t);
+        }
+    }
+
+    // bf16: both word sets of body b (columns 4b..4b+3 in scan order) of a
+    // stage, one 8-byte read per tensor and position.
+    __device__ __forceinline__ void load_quad(const unsigned char *sp, int b, PairSet &A, PairSet &B) const {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int off = rowq[r] + 8 * b;
+#pragma unroll
+            for (int t = 0; t < kTensors; ++t) {
+                const uint2 q = *reinterpret_cast<const uint2 *>(sp + off + 16 * t);
+                if constexpr (es == 2) {
+                    A[t][r] = q.x;
+                    B[t][r] = q.y;
+                }
+            }
         }
     }
 
@@ -743,12 +755,6 @@ struct ColScan {
             }
     }
 
-    // Byte offset, within a strip row's 16-byte piece, of the chunk's step k
-    // for position r (swizzled word, then the bf16 half).
-    __device__ __forceinline__ int step_byte(int k, int r) const {
-        return es == 4 ? 4 * k : 4 * ((k / 2) ^ fsw[r]) + 2 * (fwd ? (k & 1) : 1 - (k & 1));
-    }
-
     __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int col, float *ys,
                                          float *yg, bool first) const {
         const int yc = ycol(col);
@@ -767,9 +773,10 @@ struct ColScan {
 
     // Step J of body b of chunk c (launch chunk number gi; n of its CH steps
     // exist, n < CH only in the item's last chunk): steps 0-1 read word set
-    // A, steps 2-3 word set B.  B is loaded by step 0; the next body's A by
-    // step 2 (from the next chunk, waited for here, when b is the chunk's
-    // last body); `last` when chunk c ends the item.
+    // A, steps 2-3 word set B.  bf16: step 2 reads both sets of the next body
+    // (from the next chunk, waited for here, when b is the chunk's last
+    // body); fp32: B is read by step 0, the next body's A by step 2.  `last`
+    // when chunk c ends the item.
     template <int J>
     __device__ __forceinline__ void bstep(int gi, int c, int b, bool last, int n, float (&h)[R],
                                           LineW<R> (&Wb)[2], PairSet &A, PairSet &B,
@@ -780,15 +787,6 @@ struct ColScan {
         const int st = c * CH + k;  // step within the item
         recur(h, Wc);
         const bool more = b + 1 < NB || !last;   // a step follows this body's last
-        if (J == 0) load_pair(stage_ptr(gi), 2 * b + 1, B);
-        if (J == 2 && more) {
-            if (b + 1 < NB) {
-                load_pair(stage_ptr(gi), 2 * b + 2, A);
-            } else {
-                wait<0>();               // chunk gi+1 (issued when chunk gi was entered)
-                load_pair(stage_ptr(gi + 1), 0, A);
-            }
-        }
         // weights of the next step (when none follows: stale but finite
         // words, never used)
         float v[kTensors][R];
@@ -796,6 +794,28 @@ struct ColScan {
         else if (J == 1) unpack<0>(B, v);
         else if (J == 2) unpack<1>(B, v);
         else unpack<0>(A, v);
+        // word sets of the steps ahead, read after the step's last use of
+        // the set they replace
+        if constexpr (es == 2) {
+            if (J == 2 && more) {
+                if (b + 1 < NB) {
+                    load_quad(stage_ptr(gi), b + 1, A, B);
+                } else {
+                    wait<0>();           // chunk gi+1 (issued when chunk gi was entered)
+                    load_quad(stage_ptr(gi + 1), 0, A, B);
+                }
+            }
+        } else {
+            if (J == 0) load_pair(stage_ptr(gi), 2 * b + 1, B);
+            if (J == 2 && more) {
+                if (b + 1 < NB) {
+                    load_pair(stage_ptr(gi), 2 * b + 2, A);
+                } else {
+                    wait<0>();           // chunk gi+1 (issued when chunk gi was entered)
+                    load_pair(stage_ptr(gi + 1), 0, A);
+                }
+            }
+        }
         const bool bad = next_weights<PRE>(v, g, Wb[(J + 1) & 1]);
         emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
         if (!PRE) line_terms_fix(bad, v, g, Wb[(J + 1) & 1]);
@@ -824,7 +844,8 @@ struct ColScan {
                 // the item's first chunk: wait for it, weights of step 0
                 wait<1>();
                 float v[kTensors][R];
-                load_pair(stage_ptr(gi), 0, A);
+                if constexpr (es == 2) load_quad(stage_ptr(gi), 0, A, B);
+                else load_pair(stage_ptr(gi), 0, A);
                 unpack<0>(A, v);
                 first_weights<PRE>(v, g, Wb[0]);
             }
