@@ -930,10 +930,12 @@ __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem
     if (!ROW) cp_async_wait<0>();
 }
 
-// Lines of up to 96 positions keep three CTAs (12 warps) per SM: the
-// register budget is then 168 per thread.
+// Lines of up to 64 positions run four CTAs (16 warps) per SM, a budget of
+// 128 registers per thread (a few spill for fp32; measured 28 % faster on
+// 37x37 planes than three CTAs); lines of up to 96 keep three (168
+// registers: capping them at 128 was slower); longer lines two.
 template <typename T, int R, int MODE, bool PRE>
-__global__ void __launch_bounds__(kDirThreads, R <= 3 ? 3 : 2)
+__global__ void __launch_bounds__(kDirThreads, R <= 2 ? 4 : R <= 3 ? 3 : 2)
 prop2d_dir_kernel(const DirParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
