@@ -160,20 +160,6 @@ gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda, const vo
                                  int B, int Cc, int H, int W, int dirs, int share_w,
                                  gspn_dtype dtype, cudaStream_t stream);
 
-/*
- * gspn_device_status -- sticky device-side status of the current device.
- *
- * The kernels wait for their asynchronous input copies with a bounded
- * number of polls; if a copy never lands, the kernel records
- * GSPN_DEVICE_COPY_TIMEOUT here and finishes (its output is then invalid)
- * instead of hanging.  Writes the flags to *flags (0: nothing recorded) and
- * clears them if `clear` is nonzero.  Synchronous with respect to the device
- * (it reads device memory).  Returns GSPN_ERR_NULL for a NULL `flags`,
- * GSPN_ERR_CUDA if the read fails.
- */
-enum { GSPN_DEVICE_COPY_TIMEOUT = 1 };
-gspn_status gspn_device_status(unsigned int *flags, int clear);
-
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gspn_status_str(gspn_status status);
 

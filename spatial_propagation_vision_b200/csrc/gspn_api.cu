@@ -23,15 +23,7 @@ constexpr int kMaxGenericLine = 4096;   // longest line the general kernel accep
 
 }  // namespace
 
-// Device status word of the library: bit kStatusCopyTimeout is set by a
-// kernel whose bounded wait for an asynchronous copy gave up.
-__device__ unsigned int g_gspn_device_status = 0;
-
 namespace {
-
-cudaError_t status_word(unsigned int **ptr) {
-    return cudaGetSymbolAddress(reinterpret_cast<void **>(ptr), g_gspn_device_status);
-}
 
 cudaError_t device_props(DeviceProps &dp) {
     int dev = 0;
@@ -103,18 +95,6 @@ bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
 bool misaligned(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) != 0; }
 
 }  // namespace
-
-extern "C" gspn_status gspn_device_status(unsigned int *flags, int clear) {
-    if (!flags) return GSPN_ERR_NULL;
-    if (cudaMemcpyFromSymbol(flags, g_gspn_device_status, sizeof(unsigned int)) != cudaSuccess)
-        return GSPN_ERR_CUDA;
-    if (clear) {
-        const unsigned int zero = 0;
-        if (cudaMemcpyToSymbol(g_gspn_device_status, &zero, sizeof(unsigned int)) != cudaSuccess)
-            return GSPN_ERR_CUDA;
-    }
-    return GSPN_OK;
-}
 
 extern "C" const char *gspn_status_str(gspn_status s) {
     switch (s) {
@@ -222,7 +202,6 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
             pl.p.end_x = static_cast<unsigned long long>(B) * Cc * plane_bytes;
             pl.p.end_gate = 4ULL * pl.p.end_x;
             pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane_bytes;
-            if (status_word(&pl.p.status) != cudaSuccess) return GSPN_ERR_CUDA;
             const bool pre = share_w && ws;
             if (pre) {
                 // the compact mode's weights, normalised once for all channels

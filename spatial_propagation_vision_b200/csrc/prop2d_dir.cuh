@@ -85,7 +85,6 @@ struct DirParams {
     int ycol_off;               // byte offset of the column directions' output plane
     int y_pitch;                // floats per staged output row (odd, > every ycol(j), j < W)
     unsigned long long end_x, end_gate, end_wl;   // byte sizes of x, lambda/u, logits
-    unsigned int *status;       // device status word (bounded waits that gave up)
 };
 
 __device__ __forceinline__ float ex2(float x) {
