@@ -72,7 +72,8 @@ constexpr int kYSmem = 0;     // whole fp32 output plane in shared memory
 constexpr int kYBanded = 1;   // a band of output rows in shared memory, scans rerun per band
 constexpr int kYGlobal = 2;   // fp32 output accumulated in global memory (L2 atomics)
 constexpr int kYShared = 3;   // one fp32 plane in shared memory for all four directions
-                              // (shared-memory atomics): planes too large for two
+                              // (shared-memory atomics; the warps never wait for one
+                              // another before the end of a plane)
 
 struct DirParams {
     const void *x, *lam, *wl, *u;
@@ -102,14 +103,6 @@ __device__ __forceinline__ float rcp(float x) {
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-template <typename T> __device__ __forceinline__ float sload(const unsigned char *p);
-template <> __device__ __forceinline__ float sload<float>(const unsigned char *p) {
-    return *reinterpret_cast<const float *>(p);
-}
-template <> __device__ __forceinline__ float sload<__nv_bfloat16>(const unsigned char *p) {
-    return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const unsigned short *>(p)) << 16);
 }
 
 // Element offset of plane (b, c) of tensor t for direction d.
