@@ -33,6 +33,7 @@ import torch  # noqa: E402
 from spatial_propagation_vision_b200.workloads import WORKLOADS, workload_inputs  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal, reported beside the measured-peak fraction
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -373,6 +374,7 @@ def run_ours(args, w):
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic (seeded)",
         "config": config_of(w, world),
         "hbm_frac_of_measured_peak": value / world / peak,
+        "hbm_frac_of_nominal_peak": value / world / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": args.traffic if args.traffic is not None else profiled_traffic(w.name),
