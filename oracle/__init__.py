@@ -58,6 +58,8 @@ class Oracle:
         lib.oracle_prop2d_f64.restype = ctypes.c_int
         lib.oracle_prop2d_weights_f64.argtypes = [dp] + [ctypes.c_int] * 5 + [dp]
         lib.oracle_prop2d_weights_f64.restype = ctypes.c_int
+        lib.oracle_prop2d_bwd_f64.argtypes = [dp] * 5 + [ctypes.c_int] * 6 + [dp] * 4
+        lib.oracle_prop2d_bwd_f64.restype = ctypes.c_int
         self._lib = lib
 
     def prop2d(self, x, lam, wlogit, u, dirs: int = 15, share_w: int = 0) -> np.ndarray:
@@ -78,6 +80,24 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_prop2d_f64 rejected its arguments")
         return out
+
+    def prop2d_bwd(self, x, lam, wlogit, u, gy, dirs: int = 15, share_w: int = 0) -> dict:
+        """Backward of Prop2D in fp64: given gy = dL/dy, the gradients
+        {"x", "lam", "wlogit", "u"} of L, in the input layouts."""
+        x, lam, wlogit, u, gy = (_f64(t) for t in (x, lam, wlogit, u, gy))
+        B, Cc, H, W = x.shape
+        Cw = 1 if share_w else Cc
+        assert lam.shape == (B, 4, Cc, H, W) and u.shape == lam.shape, (lam.shape, u.shape)
+        assert wlogit.shape == (B, 4, Cw, 3, H, W), wlogit.shape
+        assert gy.shape == x.shape, gy.shape
+        g = {"x": np.zeros_like(x), "lam": np.zeros_like(lam), "wlogit": np.zeros_like(wlogit),
+             "u": np.zeros_like(u)}
+        rc = self._lib.oracle_prop2d_bwd_f64(
+            _ptr(x), _ptr(lam), _ptr(wlogit), _ptr(u), _ptr(gy), B, Cc, H, W, int(dirs),
+            int(bool(share_w)), _ptr(g["x"]), _ptr(g["lam"]), _ptr(g["wlogit"]), _ptr(g["u"]))
+        if rc != 0:
+            raise ValueError("oracle_prop2d_bwd_f64 rejected its arguments")
+        return g
 
     def weights(self, wlogit) -> np.ndarray:
         """Normalised tridiagonal weights [B,4,Cw,3,H,W] of a logit field (0 in off-grid slots)."""
@@ -106,3 +126,7 @@ def prop2d(x, lam, wlogit, u, dirs: int = 15, share_w: int = 0) -> np.ndarray:
 
 def weights(wlogit) -> np.ndarray:
     return default().weights(wlogit)
+
+
+def prop2d_bwd(x, lam, wlogit, u, gy, dirs: int = 15, share_w: int = 0) -> dict:
+    return default().prop2d_bwd(x, lam, wlogit, u, gy, dirs=dirs, share_w=share_w)

@@ -171,3 +171,160 @@ int oracle_prop2d_f64(const double *x, const double *lambda, const double *wlogi
     free(hcur);
     return 0;
 }
+
+/*
+ * Backward of Prop2D: the vector-Jacobian product of the forward above, in
+ * fp64.  The pages report backward timings of their kernel (Sec. 6.1
+ * "Scaling with input size, batch, and channels", Fig. 8) but print no
+ * backward formulas; what follows is the plain chain rule of the forward
+ * recurrence and normalisation, in reverse scan order.
+ *
+ * Given gy = dL/dy ([B][Cc][H][W]), for each batch b, channel c and enabled
+ * direction d, with the forward lines h_l kept:
+ *
+ *     g_l        = u_l (.) gy_l + W_{l+1}^T g_{l+1}      (adjoint of h_l; none
+ *                                                       after the last line)
+ *     du_l       = gy_l (.) h_l
+ *     dlambda_l  = g_l (.) x_l,      dx_l += g_l (.) lambda_l
+ *     dw_l(q,k)  = g_l(q) h_{l-1}(q+k-1)                 (h_{-1} = 0)
+ *
+ * and through the normalisation w_k = s_k / max(sum_k s_k, eps),
+ * s_k = sigmoid(wt_k), over the on-grid slots:
+ *
+ *     sum > eps:  ds_j = (dw_j - sum_k dw_k w_k) / sum
+ *     otherwise:  ds_j = dw_j / eps          (the clamp holds the denominator)
+ *     dwt_j = ds_j s_j (1 - s_j);   off-grid slots get 0.
+ *
+ * Readings: the derivative of max(sum, eps) is taken on the branch the
+ * forward uses (sum > eps: the sum); with share_w the gradient of the one
+ * logit field is the sum over the channels that use it.
+ *
+ * Outputs (fully written; slots of directions not in `dirs` are 0):
+ *   dx [B][Cc][H][W], dlambda [B][4][Cc][H][W], dwlogit [B][4][Cw][3][H][W],
+ *   du [B][4][Cc][H][W].
+ * Return value: 0 on success, 1 on a bad argument.
+ */
+static void normalise_parts(const double lg[3], const int valid[3], double s[3], double w[3],
+                            double *sum_out) {
+    double total = 0.0;
+    for (int k = 0; k < 3; ++k) {
+        s[k] = valid[k] ? sigmoid(lg[k]) : 0.0;
+        total += s[k];
+    }
+    normalise(lg, valid, w);
+    *sum_out = total;
+}
+
+/* Position q of line `line` of direction d (M positions per line): which
+ * neighbour slots are on the grid, their sigmoids, the normalised weights
+ * and the local sum of the sigmoids. */
+static void position_weights(const double *wlogit, size_t wplane, int H, int W, int d, int line,
+                             int q, int M, int on[3], double s[3], double w[3], double *sum) {
+    int i, j;
+    position(d, line, q, &i, &j);
+    double lg[3];
+    for (int k = 0; k < 3; ++k) {
+        int nb = q + k - 1;   /* neighbour position along the line */
+        on[k] = nb >= 0 && nb < M;
+        lg[k] = on[k] ? wlogit[at(wplane + k, H, W, i, j)] : 0.0;
+    }
+    normalise_parts(lg, on, s, w, sum);
+}
+
+int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *wlogit,
+                          const double *u, const double *gy, int B, int Cc, int H, int W,
+                          int dirs, int share_w, double *dx, double *dlambda, double *dwlogit,
+                          double *du) {
+    if (!x || !lambda || !wlogit || !u || !gy || !dx || !dlambda || !dwlogit || !du) return 1;
+    if (B < 0 || Cc < 0 || H < 0 || W < 0) return 1;
+    if (dirs < 1 || dirs > 15) return 1;
+    int Cw = share_w ? 1 : Cc;
+    size_t HW = (size_t)H * (size_t)W;
+    memset(dx, 0, (size_t)B * (size_t)Cc * HW * sizeof(double));
+    memset(dlambda, 0, (size_t)B * 4 * (size_t)Cc * HW * sizeof(double));
+    memset(du, 0, (size_t)B * 4 * (size_t)Cc * HW * sizeof(double));
+    memset(dwlogit, 0, (size_t)B * 4 * (size_t)Cw * 3 * HW * sizeof(double));
+    int maxM = H > W ? H : W;
+    /* forward lines in scan order, the adjoint line and its carry */
+    double *hist = (double *)calloc(HW + 1, sizeof(double));
+    double *adj = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    double *carry = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    double *carry_next = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    if (!hist || !adj || !carry || !carry_next) {
+        free(hist); free(adj); free(carry); free(carry_next);
+        return 1;
+    }
+
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < Cc; ++c) {
+            size_t xpl = (size_t)b * (size_t)Cc + (size_t)c;
+            for (int d = 0; d < 4; ++d) {
+                if (!(dirs & (1 << d))) continue;
+                size_t gpl = ((size_t)b * 4 + (size_t)d) * (size_t)Cc + (size_t)c;
+                size_t wpl = (((size_t)b * 4 + (size_t)d) * (size_t)Cw +
+                              (size_t)(share_w ? 0 : c)) * 3;
+                int L = d < 2 ? H : W;
+                int M = d < 2 ? W : H;
+
+                /* forward sweep, every line kept: hist[step * M + q] */
+                for (int step = 0; step < L; ++step) {
+                    int line = d % 2 ? L - 1 - step : step;   /* odd slots sweep backward */
+                    const double *prev = step > 0 ? hist + (size_t)(step - 1) * M : NULL;
+                    for (int q = 0; q < M; ++q) {
+                        int i, j, on[3];
+                        double s[3], w[3], sum;
+                        position(d, line, q, &i, &j);
+                        position_weights(wlogit, wpl, H, W, d, line, q, M, on, s, w, &sum);
+                        double v = lambda[at(gpl, H, W, i, j)] * x[at(xpl, H, W, i, j)];
+                        if (prev)
+                            for (int k = 0; k < 3; ++k)
+                                if (on[k]) v += w[k] * prev[q + k - 1];
+                        hist[(size_t)step * M + q] = v;
+                    }
+                }
+
+                /* reverse sweep of the adjoint */
+                for (int q = 0; q < M; ++q) carry[q] = 0.0;
+                for (int step = L - 1; step >= 0; --step) {
+                    int line = d % 2 ? L - 1 - step : step;   /* odd slots sweep backward */
+                    const double *hl = hist + (size_t)step * M;
+                    const double *hprv = step > 0 ? hist + (size_t)(step - 1) * M : NULL;
+                    for (int q = 0; q < M; ++q) {
+                        int i, j;
+                        position(d, line, q, &i, &j);
+                        size_t e = at(gpl, H, W, i, j);
+                        double gyv = gy[at(xpl, H, W, i, j)];
+                        adj[q] = u[e] * gyv + carry[q];
+                        du[e] = gyv * hl[q];
+                        dlambda[e] = adj[q] * x[at(xpl, H, W, i, j)];
+                        dx[at(xpl, H, W, i, j)] += adj[q] * lambda[e];
+                        carry_next[q] = 0.0;
+                    }
+                    for (int q = 0; q < M; ++q) {
+                        int i, j, on[3];
+                        double s[3], w[3], sum;
+                        position(d, line, q, &i, &j);
+                        position_weights(wlogit, wpl, H, W, d, line, q, M, on, s, w, &sum);
+                        double dw[3] = {0.0, 0.0, 0.0}, dot = 0.0;
+                        for (int k = 0; k < 3; ++k) {
+                            if (!on[k]) continue;
+                            dw[k] = hprv ? adj[q] * hprv[q + k - 1] : 0.0;
+                            dot += dw[k] * w[k];
+                            carry_next[q + k - 1] += w[k] * adj[q];
+                        }
+                        for (int k = 0; k < 3; ++k) {
+                            if (!on[k]) continue;
+                            double ds = sum > ORACLE_EPS ? (dw[k] - dot) / sum : dw[k] / ORACLE_EPS;
+                            dwlogit[at(wpl + k, H, W, i, j)] += ds * s[k] * (1.0 - s[k]);
+                        }
+                    }
+                    double *t = carry; carry = carry_next; carry_next = t;
+                }
+            }
+        }
+    free(hist);
+    free(adj);
+    free(carry);
+    free(carry_next);
+    return 0;
+}
