@@ -39,7 +39,9 @@
  * compact mode's workspace stores its normalised weights as fp16).
  *
  * Ownership: the caller owns every buffer, the workspace included.  The
- * library keeps no state between calls and allocates no memory.
+ * library allocates no memory when it is called and keeps no state between
+ * calls, except the scratch array that gspn_prop2d_fwd_noalloc uses in place
+ * of a caller workspace (a static device array, described there).
  *
  * Errors: every entry point returns a gspn_status and never aborts or traps.
  * Argument errors are detected on the host before anything is launched;
@@ -69,7 +71,9 @@ typedef enum {
     GSPN_ERR_ALIGN = 5,    /* a device pointer is not 16-byte aligned */
     GSPN_ERR_CUDA = 6,     /* the CUDA runtime reported an error */
     GSPN_ERR_DEVICE = 7,   /* the current device is not sm_100 (B200) */
-    GSPN_ERR_WORKSPACE = 8 /* workspace smaller than gspn_prop2d_workspace_bytes */
+    GSPN_ERR_WORKSPACE = 8, /* workspace smaller than gspn_prop2d_workspace_bytes */
+    GSPN_ERR_NOALLOC_LIMIT = 9 /* gspn_prop2d_fwd_noalloc: the sizes need more than
+                                  GSPN_NOALLOC_WORKSPACE_BYTES of scratch */
 } gspn_status;
 
 enum {
@@ -159,6 +163,51 @@ gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda, const vo
                                  void *d_out,
                                  int B, int Cc, int H, int W, int dirs, int share_w,
                                  gspn_dtype dtype, cudaStream_t stream);
+
+/*
+ * Size in bytes of the scratch array built into the library for
+ * gspn_prop2d_fwd_noalloc (8 MiB).
+ */
+#define GSPN_NOALLOC_WORKSPACE_BYTES (8u * 1024u * 1024u)
+
+/*
+ * gspn_prop2d_fwd_noalloc -- gspn_prop2d_fwd_ws for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a
+ * deployment variant of the compact mode.
+ *
+ * Some callers run where device allocation is not allowed: inside a host
+ * framework that owns all device memory and forbids allocating while it
+ * executes (an inference engine's per-request callback, a real-time loop
+ * with a fixed memory budget), where cudaMalloc would implicitly synchronise
+ * the device or escape the framework's accounting.  They still own x,
+ * lambda, wlogit, u and out, but cannot hand over a workspace.  This entry
+ * point takes the same arguments as gspn_prop2d_fwd and, with share_w = 1,
+ * normalises the shared weights into a scratch array compiled into the
+ * library instead of a caller workspace: a file-scope __device__ array of
+ * GSPN_NOALLOC_WORKSPACE_BYTES bytes that every GPU which loads the library
+ * holds until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * Limits and behaviour:
+ *   - share_w = 1 needs gspn_prop2d_workspace_bytes(...) bytes of scratch;
+ *     more than GSPN_NOALLOC_WORKSPACE_BYTES returns GSPN_ERR_NOALLOC_LIMIT
+ *     and launches nothing (8 MiB holds, for example, B = 8 batches of
+ *     148 x 148 bf16 grids).  With share_w = 0 no scratch is used and the
+ *     call equals gspn_prop2d_fwd.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address once (cudaGetSymbolAddress) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array, and the array keeps the
+ *     last call's contents.  Each call overwrites every weight it later
+ *     reads, so nothing has to start at zero.  Calls whose kernels overlap on
+ *     the GPU (on different streams, or from several host threads) race on
+ *     the array: order them on one stream or serialise them.
+ * Other arguments, layouts and errors as gspn_prop2d_fwd_ws.
+ */
+gspn_status gspn_prop2d_fwd_noalloc(const void *x, const void *lambda, const void *wlogit,
+                                    const void *u, int B, int Cc, int H, int W, int dirs,
+                                    int share_w, gspn_dtype dtype, void *out,
+                                    cudaStream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gspn_status_str(gspn_status status);

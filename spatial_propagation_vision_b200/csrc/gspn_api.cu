@@ -107,6 +107,9 @@ extern "C" const char *gspn_status_str(gspn_status s) {
         case GSPN_ERR_ALIGN: return "GSPN_ERR_ALIGN: device pointers must be 16-byte aligned";
         case GSPN_ERR_CUDA: return "GSPN_ERR_CUDA: CUDA runtime error";
         case GSPN_ERR_DEVICE: return "GSPN_ERR_DEVICE: the current device is not sm_100";
+        case GSPN_ERR_NOALLOC_LIMIT:
+            return "GSPN_ERR_NOALLOC_LIMIT: these sizes need more scratch than the library's "
+                   "built-in GSPN_NOALLOC_WORKSPACE_BYTES array";
     }
     return "GSPN_ERR_UNKNOWN";
 }
@@ -283,4 +286,54 @@ extern "C" gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambd
     if (cudaMemcpyAsync(h_out, d_out, nx, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return GSPN_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return GSPN_ERR_CUDA;
     return GSPN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// gspn_prop2d_fwd_noalloc: the compact mode's scratch in a library-owned
+// array, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+
+// The scratch array.  Every device that loads the library holds one copy
+// until the process exits.  In host code this name is only a host-side
+// stand-in: its device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GSPN_NOALLOC_WORKSPACE_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the first call on a device does it, with that device current).
+cudaError_t noalloc_scratch(void **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static void *addr[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" gspn_status gspn_prop2d_fwd_noalloc(const void *x, const void *lambda,
+                                               const void *wlogit, const void *u, int B, int Cc,
+                                               int H, int W, int dirs, int share_w,
+                                               gspn_dtype dtype, void *out, cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
+    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
+    if (dtype != GSPN_F32 && dtype != GSPN_BF16) return GSPN_ERR_DTYPE;
+    if (B == 0 || Cc == 0 || H == 0 || W == 0) return GSPN_OK;
+    const size_t need = workspace_bytes(B, H, W, share_w, dtype);
+    if (need > GSPN_NOALLOC_WORKSPACE_BYTES) return GSPN_ERR_NOALLOC_LIMIT;
+    void *ws = nullptr;
+    if (need > 0 && noalloc_scratch(&ws) != cudaSuccess) return GSPN_ERR_CUDA;
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, share_w, dtype, out, ws, stream);
 }

@@ -25,7 +25,10 @@ lib = ctypes.CDLL(LIB_PATH)
 GSPN_F32, GSPN_BF16 = 0, 1
 STATUS = {0: "GSPN_OK", 1: "GSPN_ERR_NULL", 2: "GSPN_ERR_SHAPE", 3: "GSPN_ERR_DIRS",
           4: "GSPN_ERR_DTYPE", 5: "GSPN_ERR_ALIGN", 6: "GSPN_ERR_CUDA", 7: "GSPN_ERR_DEVICE",
-          8: "GSPN_ERR_WORKSPACE"}
+          8: "GSPN_ERR_WORKSPACE", 9: "GSPN_ERR_NOALLOC_LIMIT"}
+
+# bytes of the library's built-in scratch array (GSPN_NOALLOC_WORKSPACE_BYTES)
+NOALLOC_WORKSPACE_BYTES = 8 * 1024 * 1024
 
 _vp, _i = ctypes.c_void_p, ctypes.c_int
 lib.gspn_prop2d_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
@@ -33,6 +36,8 @@ lib.gspn_prop2d_fwd.restype = _i
 lib.gspn_prop2d_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                                    ctypes.c_size_t, _vp]
 lib.gspn_prop2d_fwd_ws.restype = _i
+lib.gspn_prop2d_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
+lib.gspn_prop2d_fwd_noalloc.restype = _i
 lib.gspn_prop2d_workspace_bytes.argtypes = [_i] * 7
 lib.gspn_prop2d_workspace_bytes.restype = ctypes.c_size_t
 lib.gspn_prop2d_fwd_host.argtypes = [_vp] * 10 + [_i] * 7 + [_vp]
@@ -122,6 +127,38 @@ def prop2d_fwd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torc
                                         _DT[x.dtype], out.data_ptr(), workspace.data_ptr(),
                                         workspace.numel() * workspace.element_size(),
                                         _stream_handle(stream))
+    if st != 0:
+        raise GspnError(st)
+    return out
+
+
+def prop2d_fwd_noalloc(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor,
+                       u: torch.Tensor, dirs: int = 15, share_w: int = 0,
+                       out: torch.Tensor | None = None,
+                       stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Prop2D through gspn_prop2d_fwd_noalloc: the compact mode without a
+    caller workspace (the library's built-in scratch array holds the shared
+    weights), for callers that cannot allocate device memory while they run.
+    Arguments as ``prop2d_fwd``; only ``out`` may be allocated here, and only
+    when it is not given."""
+    B, Cc, H, W = _dims(x)
+    if x.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    Cw = 1 if share_w else Cc
+    dev = x.device
+    _check("x", x, (B, Cc, H, W), x.dtype, dev)
+    _check("lam", lam, (B, 4, Cc, H, W), x.dtype, dev)
+    _check("u", u, (B, 4, Cc, H, W), x.dtype, dev)
+    _check("wlogit", wlogit, (B, 4, Cw, 3, H, W), x.dtype, dev)
+    if out is None:
+        out = torch.empty((B, Cc, H, W), dtype=x.dtype, device=dev)
+    _check("out", out, (B, Cc, H, W), x.dtype, dev)
+    with torch.cuda.device(dev):
+        st = lib.gspn_prop2d_fwd_noalloc(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(),
+                                         u.data_ptr(), B, Cc, H, W, int(dirs), int(share_w),
+                                         _DT[x.dtype], out.data_ptr(), _stream_handle(stream))
     if st != 0:
         raise GspnError(st)
     return out
