@@ -60,6 +60,8 @@ class Oracle:
         lib.oracle_prop2d_weights_f64.restype = ctypes.c_int
         lib.oracle_prop2d_bwd_f64.argtypes = [dp] * 5 + [ctypes.c_int] * 6 + [dp] * 4
         lib.oracle_prop2d_bwd_f64.restype = ctypes.c_int
+        lib.oracle_prop2d_ex_f64.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 7 + [dp]
+        lib.oracle_prop2d_ex_f64.restype = ctypes.c_int
         self._lib = lib
 
     def prop2d(self, x, lam, wlogit, u, dirs: int = 15, share_w: int = 0) -> np.ndarray:
@@ -79,6 +81,23 @@ class Oracle:
                                          B, Cc, H, W, int(dirs), int(bool(share_w)), _ptr(out))
         if rc != 0:
             raise ValueError("oracle_prop2d_f64 rejected its arguments")
+        return out
+
+    def prop2d_ex(self, x, lam, wlogit, u, dirs: int = 15, gate_dirs: int = 4,
+                  w_groups: int | None = None) -> np.ndarray:
+        """Forward with shared gates / grouped logits: lam, u [B,gate_dirs,Cc,H,W]
+        (gate_dirs 4 or 1); wlogit [B,4,G,3,H,W], channel c using field
+        c // (Cc // G) (G = w_groups, default Cc)."""
+        x, lam, wlogit, u = (_f64(t) for t in (x, lam, wlogit, u))
+        B, Cc, H, W = x.shape
+        G = Cc if w_groups is None else int(w_groups)
+        assert lam.shape == (B, gate_dirs, Cc, H, W) and u.shape == lam.shape, lam.shape
+        assert wlogit.shape == (B, 4, G, 3, H, W), wlogit.shape
+        out = np.zeros((B, Cc, H, W), dtype=np.float64)
+        rc = self._lib.oracle_prop2d_ex_f64(_ptr(x), _ptr(lam), _ptr(wlogit), _ptr(u), B, Cc, H,
+                                            W, int(dirs), int(gate_dirs), G, _ptr(out))
+        if rc != 0:
+            raise ValueError("oracle_prop2d_ex_f64 rejected its arguments")
         return out
 
     def prop2d_bwd(self, x, lam, wlogit, u, gy, dirs: int = 15, share_w: int = 0) -> dict:
@@ -130,3 +149,7 @@ def weights(wlogit) -> np.ndarray:
 
 def prop2d_bwd(x, lam, wlogit, u, gy, dirs: int = 15, share_w: int = 0) -> dict:
     return default().prop2d_bwd(x, lam, wlogit, u, gy, dirs=dirs, share_w=share_w)
+
+
+def prop2d_ex(x, lam, wlogit, u, dirs: int = 15, gate_dirs: int = 4, w_groups=None) -> np.ndarray:
+    return default().prop2d_ex(x, lam, wlogit, u, dirs=dirs, gate_dirs=gate_dirs, w_groups=w_groups)

@@ -328,3 +328,74 @@ int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *w
     free(carry_next);
     return 0;
 }
+
+/*
+ * Gate- and weight-sharing variants of the forward (the pages' "share w_i
+ * across channels in all modules", Sec. 6.2 "Image classification", and the
+ * channel-shared weights of Sec. 4.2, generalised):
+ *
+ *   gate_dirs = 4: lambda and u hold one plane per direction, [B][4][Cc][H][W];
+ *   gate_dirs = 1: one lambda and one u plane serve all four directions,
+ *                  [B][1][Cc][H][W];
+ *   w_groups  = G (G divides Cc): the logits hold G fields per (batch,
+ *                  direction), [B][4][G][3][H][W]; channel c uses field
+ *                  c / (Cc / G).  G = Cc is per-channel, G = 1 is share_w.
+ *
+ * Everything else is the forward above.  Return value: 0 on success, 1 on a
+ * bad argument.
+ */
+int oracle_prop2d_ex_f64(const double *x, const double *lambda, const double *wlogit,
+                         const double *u, int B, int Cc, int H, int W, int dirs,
+                         int gate_dirs, int w_groups, double *out) {
+    if (!x || !lambda || !wlogit || !u || !out) return 1;
+    if (B < 0 || Cc < 0 || H < 0 || W < 0) return 1;
+    if (dirs < 1 || dirs > 15) return 1;
+    if (gate_dirs != 1 && gate_dirs != 4) return 1;
+    if (w_groups < 1 || (Cc > 0 && Cc % w_groups != 0)) return 1;
+    int per_group = Cc > 0 ? Cc / w_groups : 1;
+    int maxM = H > W ? H : W;
+    double *before = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    double *after = (double *)calloc((size_t)maxM + 1, sizeof(double));
+    if (!before || !after) { free(before); free(after); return 1; }
+
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < Cc; ++c) {
+            size_t xo = (size_t)b * (size_t)Cc + (size_t)c;
+            for (int i = 0; i < H; ++i)
+                for (int j = 0; j < W; ++j) out[at(xo, H, W, i, j)] = 0.0;
+            for (int d = 0; d < 4; ++d) {
+                if (!(dirs & (1 << d))) continue;
+                /* lambda / u plane: the direction's own, or the one shared plane */
+                size_t go = ((size_t)b * (size_t)gate_dirs + (size_t)(gate_dirs == 4 ? d : 0)) *
+                                (size_t)Cc + (size_t)c;
+                /* logit field of the channel's group */
+                size_t wo = (((size_t)b * 4 + (size_t)d) * (size_t)w_groups +
+                             (size_t)(c / per_group)) * 3;
+                int L = d < 2 ? H : W;
+                int M = d < 2 ? W : H;
+                for (int q = 0; q < M; ++q) before[q] = 0.0;
+                for (int step = 0; step < L; ++step) {
+                    int line = d % 2 ? L - 1 - step : step;
+                    for (int q = 0; q < M; ++q) {
+                        int i, j, on[3];
+                        double s[3], w[3], sum;
+                        position(d, line, q, &i, &j);
+                        position_weights(wlogit, wo, H, W, d, line, q, M, on, s, w, &sum);
+                        double v = 0.0;
+                        for (int k = 0; k < 3; ++k)
+                            if (on[k]) v += w[k] * before[q + k - 1];
+                        after[q] = v + lambda[at(go, H, W, i, j)] * x[at(xo, H, W, i, j)];
+                    }
+                    for (int q = 0; q < M; ++q) {
+                        int i, j;
+                        position(d, line, q, &i, &j);
+                        out[at(xo, H, W, i, j)] += u[at(go, H, W, i, j)] * after[q];
+                    }
+                    double *t = before; before = after; after = t;
+                }
+            }
+        }
+    free(before);
+    free(after);
+    return 0;
+}
