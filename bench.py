@@ -60,11 +60,20 @@ def kernel_sources_sha() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    if it was captured on the current kernel sources; else None."""
+KERNEL_OF_PATH = {"pair": "prop2d_pair_kernel", "dir": "prop2d_dir_kernel",
+                  "dir-shared": "prop2d_dir_kernel", "dir-yglobal": "prop2d_dir_kernel",
+                  "dir-banded": "prop2d_dir_kernel", "generic": "prop2d_generic_kernel"}
+
+
+def profile_path(kernel: str, workload: str) -> str:
+    return os.path.join(ROOT, "profiles", f"{kernel.replace('_kernel', '')}_{workload}.md")
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on
+    this workload, if it was captured on the current kernel sources; else None."""
     import re
-    path = os.path.join(ROOT, "profiles", f"prop2d_dir_{workload}.md")
+    path = profile_path(kernel, workload)
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -115,7 +124,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -141,18 +150,18 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def window(self, a, b):
+        """Statistics of the samples taken between marks `a` and `b`."""
         rows = []
         for ts, line in self.samples:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             rows.append((ts, parts))
-        inwin = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
-        use = inwin or rows[-3:]
+        t0, t1 = getattr(self, a, None), getattr(self, b, None)
+        use = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
         if not use:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
-                    "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
 
         def num(s):
             try:
@@ -165,8 +174,27 @@ class ClockSampler:
         reasons = sorted({n for _, p in use for n, v in zip(names, p[5:9]) if v.strip() == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(inwin),
+                "reasons": reasons, "samples": len(use),
                 "power_w_max": max((num(p[3]) or 0.0) for _, p in use)}
+
+    def summary(self):
+        """Clocks of the timed region; when it was too short for a sample
+        (20 ms polling), those of the load window run just before it, which
+        is said so in `source`."""
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0, "source": "none"}
+        timed = self.window("t0", "t1")
+        load = self.window("l0", "l1")
+        if timed["samples"]:
+            out = dict(timed, source="timed region")
+        else:
+            out = dict(load, source="no sample in the timed region (shorter than the 20 ms "
+                                    "polling interval); load window of the same call run for "
+                                    "about 1 s just before it")
+        out["timed_region_samples"] = timed["samples"]
+        out["load_window"] = load
+        return out
 
 
 # ----------------------------------------------------------------------------
@@ -302,6 +330,19 @@ def run_ours(args, w):
 
     sampler = ClockSampler(dev.index)
     sampler.start()
+    # load window: the same call for about 1 s (untimed), sampled for clocks
+    # in case the timed region below is shorter than the polling interval
+    torch.cuda.synchronize(dev)
+    sampler.mark("l0")
+    t_load = time.time()
+    with torch.cuda.stream(stream):
+        while time.time() - t_load < 1.0:
+            for _ in range(20):
+                if flush is not None:
+                    flush.fill_(1.0)
+                call()
+            torch.cuda.synchronize(dev)
+    sampler.mark("l1")
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     if world > 1:
@@ -366,6 +407,8 @@ def run_ours(args, w):
 
     peak, peak_kind = peaks()
     achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
+    kernel = KERNEL_OF_PATH.get(info["path"], info["path"])
+    traffic = args.traffic if args.traffic is not None else profiled_traffic(kernel, w.name)
     value = job_value(nbytes, world, step_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -377,12 +420,13 @@ def run_ours(args, w):
         "hbm_frac_of_nominal_peak": value / world / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": args.traffic if args.traffic is not None else profiled_traffic(w.name),
+                     "traffic": traffic,
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch "
-                                       f"(profiles/prop2d_dir_{w.name}.md, same kernel sources) or null",
+                                       f"({os.path.relpath(profile_path(kernel, w.name), ROOT)}, "
+                                       "same kernel sources) or null",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "prop2d_dir_kernel", "avg_launch_ms": avg_kernel_ms},
+                     "kernel": kernel, "avg_launch_ms": avg_kernel_ms},
         "e2e": {"value": job_value(nbytes, world, e2e_ms * 1e-3), "unit": "GB/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "gspn_prop2d_fwd_host (pinned host buffers)"},

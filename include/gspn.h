@@ -72,8 +72,10 @@ typedef enum {
     GSPN_ERR_CUDA = 6,     /* the CUDA runtime reported an error */
     GSPN_ERR_DEVICE = 7,   /* the current device is not sm_100 (B200) */
     GSPN_ERR_WORKSPACE = 8, /* workspace smaller than gspn_prop2d_workspace_bytes */
-    GSPN_ERR_NOALLOC_LIMIT = 9 /* gspn_prop2d_fwd_noalloc: the sizes need more than
-                                  GSPN_NOALLOC_WORKSPACE_BYTES of scratch */
+    GSPN_ERR_NOALLOC_LIMIT = 9, /* gspn_prop2d_fwd_noalloc: the sizes need more than
+                                   GSPN_NOALLOC_WORKSPACE_BYTES of scratch */
+    GSPN_ERR_SHARING = 10  /* gspn_prop2d_fwd_ex: gate_dirs not 1 or 4, or w_groups not a
+                              divisor of Cc */
 } gspn_status;
 
 enum {
@@ -108,6 +110,28 @@ gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const void *wlogi
                             const void *u, int B, int Cc, int H, int W, int dirs,
                             int share_w, gspn_dtype dtype, void *out,
                             cudaStream_t stream);
+
+/*
+ * gspn_prop2d_fwd_ex -- gspn_prop2d_fwd with the gates and the logits shared
+ * more widely (Sec. 4.2 "Channel-shared weights and the attention view";
+ * Sec. 6.2 "Image classification", which shares w_i across channels in all
+ * modules).
+ *
+ * gate_dirs : 4 -> lambda and u hold one plane per direction, [B][4][Cc][H][W]
+ *                  (as gspn_prop2d_fwd);
+ *             1 -> one lambda plane and one u plane serve all four
+ *                  directions: lambda, u are [B][1][Cc][H][W].
+ * w_groups  : G, a divisor of Cc: wlogit is [B][4][G][3][H][W] and channel c
+ *             uses logit field c / (Cc / G).  G = Cc is gspn_prop2d_fwd's
+ *             share_w = 0, G = 1 its share_w = 1.
+ * Other arguments as gspn_prop2d_fwd.  Returns GSPN_ERR_SHARING for a
+ * gate_dirs other than 1 or 4 or a w_groups that does not divide Cc (w_groups
+ * < 1 included), before anything is launched.
+ */
+gspn_status gspn_prop2d_fwd_ex(const void *x, const void *lambda, const void *wlogit,
+                               const void *u, int B, int Cc, int H, int W, int dirs,
+                               int gate_dirs, int w_groups, gspn_dtype dtype, void *out,
+                               cudaStream_t stream);
 
 /*
  * gspn_prop2d_workspace_bytes -- size of the workspace gspn_prop2d_fwd_ws

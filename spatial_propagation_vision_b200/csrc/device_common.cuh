@@ -10,23 +10,32 @@ namespace gspn {
 // ---------------------------------------------------------------------------
 // element types
 // ---------------------------------------------------------------------------
-template <typename T> struct Elem;
-template <> struct Elem<float> {
-    static __device__ __forceinline__ float load(const float *p) { return *p; }
-    static __device__ __forceinline__ float to_f(float v) { return v; }
-    static __device__ __forceinline__ float from_f(float v) { return v; }
-};
-template <> struct Elem<__nv_bfloat16> {
-    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
-    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
-};
-
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
     return __float2bfloat16_rn(v);
+}
+
+// ---------------------------------------------------------------------------
+// hardware approximations: 2^x and 1/x (flush-to-zero), byte permutation
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// Byte permutation of (x, 0): bf16 half of a word -> fp32 bits.
+__device__ __forceinline__ uint32_t prmt0(uint32_t x, uint32_t sel) {
+    uint32_t y;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(x), "r"(sel));
+    return y;
 }
 
 // ---------------------------------------------------------------------------

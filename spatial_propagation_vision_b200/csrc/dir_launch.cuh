@@ -9,10 +9,8 @@ namespace gspn_host {
 template <typename T, int R, int MODE, bool PRE>
 cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t stream, LaunchInfo &li) {
     auto kern = gspn::prop2d_dir_kernel<T, R, MODE, PRE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
-    if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kDirThreads, pl.smem);
+    cudaError_t e = kernel_occupancy(reinterpret_cast<const void *>(kern), gspn::kDirThreads, pl.smem, per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = static_cast<long long>(dp.sms) * per_sm;

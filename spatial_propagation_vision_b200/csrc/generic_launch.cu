@@ -21,10 +21,8 @@ static cudaError_t launch_generic_t(const gspn::GenericParams &gp0, const Device
     gp.n_items = gp.B * gp.Cc * gp.bands;
     const int smem = round_up(band_rows * YP * 4, 16) + hbytes;
     auto kern = gspn::prop2d_generic_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gspn::kGenericThreads, smem);
+    cudaError_t e = kernel_occupancy(reinterpret_cast<const void *>(kern), gspn::kGenericThreads, smem, per_sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = static_cast<long long>(dp.sms) * per_sm;

@@ -18,6 +18,13 @@ using namespace gspn_host;
 
 thread_local LaunchInfo g_last;
 
+// How the gate and logit tensors are shared: direction slots of lambda and
+// u (4, or 1 shared by all directions) and logit fields per (batch,
+// direction) (Cc per channel; 1 the compact mode's shared field).
+struct Sharing {
+    int gate_dirs, w_groups;
+};
+
 constexpr int kMaxDirLine = 256;        // longest line (H or W) the direction kernel holds in registers
 constexpr int kMaxGenericLine = 4096;   // longest line the general kernel accepts
 
@@ -42,6 +49,47 @@ cudaError_t device_props(DeviceProps &dp) {
     if (dev < 64) { cache[dev] = dp; have[dev] = true; }
     return cudaSuccess;
 }
+
+}  // namespace
+
+namespace gspn_host {
+
+cudaError_t kernel_occupancy(const void *kernel, int threads, int smem, int &per_sm) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    struct Entry { int dev; const void *kernel; int threads, smem, per_sm; };
+    static std::mutex mu;
+    static Entry cache[256];
+    static int n = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i) {
+        const Entry &c = cache[i];
+        if (c.dev == dev && c.kernel == kernel && c.threads == threads && c.smem == smem) {
+            per_sm = c.per_sm;
+            return cudaSuccess;
+        }
+    }
+    // the limit is per kernel: raise it once to the device maximum (never
+    // lower it, which would fail a later launch with more shared memory)
+    bool raised = false;
+    for (int i = 0; i < n && !raised; ++i) raised = cache[i].dev == dev && cache[i].kernel == kernel;
+    if (!raised) {
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e != cudaSuccess) return e;
+    }
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (n < 256) cache[n++] = Entry{dev, kernel, threads, smem, per_sm};
+    return cudaSuccess;
+}
+
+}  // namespace gspn_host
+
+namespace {
 
 // Shared-memory plan for output mode `mode` so that one CTA fits `cap`
 // bytes.  Output modes: 0, fp32 output planes in shared memory (one for the
@@ -107,6 +155,8 @@ extern "C" const char *gspn_status_str(gspn_status s) {
         case GSPN_ERR_ALIGN: return "GSPN_ERR_ALIGN: device pointers must be 16-byte aligned";
         case GSPN_ERR_CUDA: return "GSPN_ERR_CUDA: CUDA runtime error";
         case GSPN_ERR_DEVICE: return "GSPN_ERR_DEVICE: the current device is not sm_100";
+        case GSPN_ERR_SHARING:
+            return "GSPN_ERR_SHARING: gate_dirs must be 1 or 4 and w_groups a divisor of Cc";
         case GSPN_ERR_NOALLOC_LIMIT:
             return "GSPN_ERR_NOALLOC_LIMIT: these sizes need more scratch than the library's "
                    "built-in GSPN_NOALLOC_WORKSPACE_BYTES array";
@@ -138,25 +188,87 @@ using DirLaunch = cudaError_t (*)(int, const DirPlan &, const DeviceProps &, cud
 // The direction kernel variant for (element size, output path, weights
 // normalised ahead).
 DirLaunch dir_variant(int es, const DirPlan &pl, bool pre) {
-    const bool banded = pl.p.bands > 1;
     if (es == 4) {
+        // (fp32 never needs bands: global accumulation always fits)
         if (pl.y_global) return pre ? launch_dir_f32_global_pre : launch_dir_f32_global;
         if (pl.y_shared) return pre ? launch_dir_f32_shared_pre : launch_dir_f32_shared;
-        if (banded) return pre ? launch_dir_f32_banded_pre : launch_dir_f32_banded;
         return pre ? launch_dir_f32_smem_pre : launch_dir_f32_smem;
     }
     if (pl.y_shared) return pre ? launch_dir_bf16_shared_pre : launch_dir_bf16_shared;
     return pre ? launch_dir_bf16_banded_pre : launch_dir_bf16_banded;
 }
 
-// gspn_prop2d_fwd with an optional workspace (compact mode only: the
-// weights are then normalised once into it and read by every channel).
+// Lines of up to kMaxPairLine positions run on the sweep-pair kernel, with
+// RP pairs and NS single positions per lane chosen from the longer side:
+// capacity 32 RP + 16 NS.
+constexpr int kMaxPairLine = 128;
+
+// Sweep-pair kernel (prop2d_pair.cuh) when the shape suits it: both sides
+// 2..128, rows at least as long as the lanes' pair blocks (their words are
+// read straight from global memory), bf16 rows of even width (4-byte aligned
+// pair words), every tensor under 4 GiB (32-bit byte offsets), and the two
+// output planes and the column rings in shared memory.  `taken` tells
+// whether it was launched.
+cudaError_t try_pair(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
+                     int Cc, int H, int W, int dirs, Sharing sh, int es, void *out,
+                     const DeviceProps &dp, cudaStream_t stream, bool &taken) {
+    taken = false;
+    const int mx = H > W ? H : W;
+    if (H < 2 || W < 2 || mx > kMaxPairLine || (es == 2 && W % 2)) return cudaSuccess;
+    const int bucket = (mx + 15) / 16 - 1;           // 0 .. 7
+    const int RP = bucket / 2, NS = bucket % 2 + 1;  // capacity 32 RP + 16 NS >= mx
+    if (W < 32 * RP) return cudaSuccess;
+    const unsigned long long plane = static_cast<unsigned long long>(H) * W * es;
+    const unsigned long long xb = static_cast<unsigned long long>(B) * Cc * plane;
+    const unsigned long long gb = static_cast<unsigned long long>(sh.gate_dirs) * xb;
+    const unsigned long long wb = static_cast<unsigned long long>(B) * 4 * sh.w_groups * 3 * plane;
+    if (gb >= (1ULL << 32) || wb >= (1ULL << 32)) return cudaSuccess;
+    // output line pitch: at least the capacity, a multiple of 4 floats with
+    // an odd number of 16-byte units (conflict-free transposed reads)
+    const int cap = 32 * RP + 16 * NS;
+    int yp = round_up(cap, 4);
+    if ((yp / 4) % 2 == 0) yp += 4;
+    const int grp = RP > 0 ? 2 * RP : 1;
+    const int stage = round_up(4 * (H * gspn::kPairRowWords + ((H + grp - 1) / grp) * gspn::kPairSkewWords), 16);
+    // output planes of the I/O element type (bf16 partial sums for bf16 inputs)
+    const int q_off = round_up(H * yp * es, 16);
+    const int ring_off = q_off + round_up(W * yp * es, 16);
+    const int smem = ring_off + 2 * gspn::kPairStages * stage;
+    if (smem > dp.smem_optin) return cudaSuccess;
+    gspn::PairParams pp{};
+    pp.x = static_cast<const char *>(x);
+    pp.lam = static_cast<const char *>(lambda);
+    pp.u = static_cast<const char *>(u);
+    pp.wl0 = static_cast<const char *>(wlogit);
+    pp.wl1 = pp.wl0 + plane;
+    pp.wl2 = pp.wl0 + 2 * plane;
+    pp.out = out;
+    pp.B = B; pp.Cc = Cc; pp.H = H; pp.W = W; pp.dirs = dirs;
+    pp.gate_dirs = sh.gate_dirs;
+    pp.w_groups = sh.w_groups;
+    pp.w_cpg = Cc / sh.w_groups;
+    pp.n_items = B * Cc;
+    pp.yp = yp;
+    pp.q_off = q_off;
+    pp.ring_off = ring_off;
+    pp.stage_bytes = stage;
+    pp.x_bytes = static_cast<unsigned int>(xb);
+    pp.g_bytes = static_cast<unsigned int>(gb);
+    pp.w_bytes = static_cast<unsigned int>(wb);
+    taken = true;
+    return es == 2 ? launch_pair_bf16(RP, NS, pp, smem, dp, stream, g_last)
+                   : launch_pair_f32(RP, NS, pp, smem, dp, stream, g_last);
+}
+
+// Prop2D with the callers' sharing of gates and logits, and an optional
+// workspace (one logit field per (batch, direction) only: the weights are
+// then normalised once into it and read by every channel).  The callers
+// check `dirs` and the sharing arguments.
 gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
-                       int Cc, int H, int W, int dirs, int share_w, gspn_dtype dtype, void *out,
+                       int Cc, int H, int W, int dirs, Sharing sh, gspn_dtype dtype, void *out,
                        void *ws, cudaStream_t stream) {
     g_last = LaunchInfo{};
     if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
-    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
     if (dtype != GSPN_F32 && dtype != GSPN_BF16) return GSPN_ERR_DTYPE;
     if (B == 0 || Cc == 0 || H == 0 || W == 0) return GSPN_OK;
     if (!x || !lambda || !wlogit || !u || !out) return GSPN_ERR_NULL;
@@ -175,13 +287,22 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
 
     const int es = dtype == GSPN_BF16 ? 2 : 4;
     cudaError_t err = cudaSuccess;
+    const bool pre = sh.w_groups == 1 && ws;
+    if (!pre) {
+        bool taken = false;
+        err = try_pair(x, lambda, wlogit, u, B, Cc, H, W, dirs, sh, es, out, dp, stream, taken);
+        if (taken) return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+    }
     // bf16 rows of even width keep every row and span 4-byte aligned
     const bool dir_ok = maxline <= kMaxDirLine && H >= 2 && W >= 2 && (es == 4 || (W % 2 == 0));
     if (dir_ok) {
         const int R = (maxline + 31) / 32;
         DirPlan pl;
         pl.p.x = x; pl.p.lam = lambda; pl.p.wl = wlogit; pl.p.u = u; pl.p.out = out;
-        pl.p.B = B; pl.p.Cc = Cc; pl.p.H = H; pl.p.W = W; pl.p.dirs = dirs; pl.p.share_w = share_w;
+        pl.p.B = B; pl.p.Cc = Cc; pl.p.H = H; pl.p.W = W; pl.p.dirs = dirs;
+        pl.p.gate_dirs = sh.gate_dirs;
+        pl.p.w_groups = sh.w_groups;
+        pl.p.w_cpg = Cc / sh.w_groups;
         // Output modes in order of preference (the last reruns the scans per
         // band); within a mode, the most CTAs per SM that fit.
         const int caps[4] = {dp.smem_per_sm / 4 - 1024, dp.smem_per_sm / 3 - 1024,
@@ -189,9 +310,9 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
         bool fit = false;
         // bf16: one plane with shared atomics (the four directions run
         // uncoupled until the end of an item), else bands; fp32: two planes
-        // (atomic-free), one plane, global atomics, else bands
-        const int order_bf16[2] = {3, 2}, order_f32[4] = {0, 3, 1, 2};
-        const int n_order = es == 2 ? 2 : 4;
+        // (atomic-free), one plane, else global atomics (which always fit)
+        const int order_bf16[2] = {3, 2}, order_f32[3] = {0, 3, 1};
+        const int n_order = es == 2 ? 2 : 3;
         for (int oi = 0; oi < n_order && !fit; ++oi) {
             const int mode = es == 2 ? order_bf16[oi] : order_f32[oi];
             for (int ci = 0; ci < 4 && !fit; ++ci) {
@@ -203,9 +324,8 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
             pl.p.n_items = B * Cc * pl.p.bands;
             const unsigned long long plane_bytes = static_cast<unsigned long long>(HW) * es;
             pl.p.end_x = static_cast<unsigned long long>(B) * Cc * plane_bytes;
-            pl.p.end_gate = 4ULL * pl.p.end_x;
-            pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane_bytes;
-            const bool pre = share_w && ws;
+            pl.p.end_gate = static_cast<unsigned long long>(sh.gate_dirs) * pl.p.end_x;
+            pl.p.end_wl = static_cast<unsigned long long>(B) * 4 * sh.w_groups * 3 * plane_bytes;
             if (pre) {
                 // the compact mode's weights, normalised once for all channels
                 gspn::NormParams np{wlogit, ws, B, H, W, dirs};
@@ -219,7 +339,10 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
     }
     GenericParams gp{};
     gp.x = x; gp.lam = lambda; gp.wl = wlogit; gp.u = u; gp.out = out;
-    gp.B = B; gp.Cc = Cc; gp.H = H; gp.W = W; gp.dirs = dirs; gp.share_w = share_w;
+    gp.B = B; gp.Cc = Cc; gp.H = H; gp.W = W; gp.dirs = dirs;
+    gp.gate_dirs = sh.gate_dirs;
+    gp.w_groups = sh.w_groups;
+    gp.w_cpg = Cc / sh.w_groups;
     bool fits = false;
     err = launch_generic(gp, es == 2, dp, stream, fits, g_last);
     if (!fits) return GSPN_ERR_SHAPE;
@@ -232,7 +355,22 @@ extern "C" gspn_status gspn_prop2d_fwd(const void *x, const void *lambda, const 
                                        const void *u, int B, int Cc, int H, int W, int dirs,
                                        int share_w, gspn_dtype dtype, void *out,
                                        cudaStream_t stream) {
-    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, share_w, dtype, out, nullptr, stream);
+    g_last = LaunchInfo{};
+    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{4, share_w ? 1 : Cc}, dtype,
+                      out, nullptr, stream);
+}
+
+extern "C" gspn_status gspn_prop2d_fwd_ex(const void *x, const void *lambda, const void *wlogit,
+                                          const void *u, int B, int Cc, int H, int W, int dirs,
+                                          int gate_dirs, int w_groups, gspn_dtype dtype, void *out,
+                                          cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (dirs < 1 || dirs > 15) return GSPN_ERR_DIRS;
+    if ((gate_dirs != 1 && gate_dirs != 4) || w_groups < 1 || (Cc > 0 && Cc % w_groups != 0))
+        return GSPN_ERR_SHARING;
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{gate_dirs, w_groups}, dtype,
+                      out, nullptr, stream);
 }
 
 extern "C" size_t gspn_prop2d_workspace_bytes(int B, int Cc, int H, int W, int dirs, int share_w,
@@ -256,8 +394,8 @@ extern "C" gspn_status gspn_prop2d_fwd_ws(const void *x, const void *lambda, con
         if (workspace_size < need) return GSPN_ERR_WORKSPACE;
         if (misaligned(workspace)) return GSPN_ERR_ALIGN;
     }
-    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, share_w, dtype, out,
-                      need > 0 ? workspace : nullptr, stream);
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{4, share_w ? 1 : Cc}, dtype,
+                      out, need > 0 ? workspace : nullptr, stream);
 }
 
 extern "C" gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda,
@@ -335,5 +473,6 @@ extern "C" gspn_status gspn_prop2d_fwd_noalloc(const void *x, const void *lambda
     if (need > GSPN_NOALLOC_WORKSPACE_BYTES) return GSPN_ERR_NOALLOC_LIMIT;
     void *ws = nullptr;
     if (need > 0 && noalloc_scratch(&ws) != cudaSuccess) return GSPN_ERR_CUDA;
-    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, share_w, dtype, out, ws, stream);
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{4, share_w ? 1 : Cc}, dtype,
+                      out, ws, stream);
 }

@@ -10,6 +10,7 @@
 #include "prop2d_dir.cuh"
 #include "prop2d_generic.cuh"
 #include "prop2d_norm.cuh"
+#include "prop2d_pair.cuh"
 
 namespace gspn_host {
 
@@ -37,8 +38,6 @@ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 // normalised in the scan or ahead: _pre); R is the positions per lane (1..8).
 cudaError_t launch_dir_f32_smem(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_smem_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
-cudaError_t launch_dir_f32_banded(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
-cudaError_t launch_dir_f32_banded_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_global(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_global_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_f32_shared(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
@@ -47,6 +46,17 @@ cudaError_t launch_dir_bf16_banded(int R, const DirPlan &pl, const DeviceProps &
 cudaError_t launch_dir_bf16_banded_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_shared(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_shared_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+
+// Sweep-pair kernel: RP position pairs and NS single positions per lane.
+cudaError_t launch_pair_bf16(int RP, int NS, const gspn::PairParams &pp, int smem,
+                             const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_pair_f32(int RP, int NS, const gspn::PairParams &pp, int smem,
+                            const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+
+// Resident CTAs per SM of `kernel` with `smem` bytes of dynamic shared
+// memory; sets the kernel's shared-memory limit.  Both are cached per
+// (device, kernel, smem), so repeated calls make no runtime queries.
+cudaError_t kernel_occupancy(const void *kernel, int threads, int smem, int &per_sm);
 
 // Normalised weights of the compact mode into the workspace (one launch).
 cudaError_t launch_norm(const gspn::NormParams &np, bool bf16, const DeviceProps &dp, cudaStream_t s);

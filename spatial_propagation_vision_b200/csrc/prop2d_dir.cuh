@@ -78,7 +78,9 @@ constexpr int kYShared = 3;   // one fp32 plane in shared memory for all four di
 struct DirParams {
     const void *x, *lam, *wl, *u;
     void *out;
-    int B, Cc, H, W, dirs, share_w;
+    int B, Cc, H, W, dirs;
+    int gate_dirs;              // direction slots of lambda and u: 4, or 1 shared by all directions
+    int w_groups, w_cpg;        // logit fields per (batch, direction) and channels per field
     int n_items, bands, band_rows;
     int stage_col;              // bytes per column ring stage
     int ring[4];                // byte offset of column direction d's ring (-1: none)
@@ -88,30 +90,14 @@ struct DirParams {
     unsigned long long end_x, end_gate, end_wl;   // byte sizes of x, lambda/u, logits
 };
 
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// Byte permutation of (x, 0): bf16 half of a word -> fp32 bits.
-__device__ __forceinline__ uint32_t prmt0(uint32_t x, uint32_t sel) {
-    uint32_t y;
-    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(x), "r"(sel));
-    return y;
-}
-__device__ __forceinline__ float rcp(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // Element offset of plane (b, c) of tensor t for direction d.
 __device__ __forceinline__ size_t dir_plane(const DirParams &p, int b, int c, int d, int t) {
     const size_t HW = static_cast<size_t>(p.H) * p.W;
     if (t == 5) return (static_cast<size_t>(b) * p.Cc + c) * HW;
-    if (t < 2) return ((static_cast<size_t>(b) * 4 + d) * p.Cc + c) * HW;
-    const int Cw = p.share_w ? 1 : p.Cc;
-    return ((((static_cast<size_t>(b) * 4 + d) * Cw + (p.share_w ? 0 : c)) * 3) + (t - 2)) * HW;
+    if (t < 2)
+        return ((static_cast<size_t>(b) * p.gate_dirs + (p.gate_dirs == 4 ? d : 0)) * p.Cc + c) * HW;
+    return ((((static_cast<size_t>(b) * 4 + d) * p.w_groups + c / p.w_cpg) * 3) + (t - 2)) * HW;
 }
 
 __device__ __forceinline__ const char *dir_tensor(const DirParams &p, int t) {
@@ -214,9 +200,14 @@ __device__ __forceinline__ void line_weights_plain_v(const float (&v)[kTensors][
     constexpr float nl2e = -1.4426950408889634f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        const float s0 = rcp(1.0f + ex2(v[2][r] * nl2e)) * g.m0[r];
-        const float s1 = rcp(1.0f + ex2(v[3][r] * nl2e));
-        const float s2 = rcp(1.0f + ex2(v[4][r] * nl2e)) * g.m2[r];
+        // off-grid slots are selected away (their logits may be anything,
+        // NaN included, and must not reach the weights)
+        // (positions past the line's end read another position's inputs,
+        // off-grid slots included, and take no weight at all)
+        const bool on = g.valid[r];
+        const float s0 = on && g.m0[r] != 0.0f ? rcp(1.0f + ex2(v[2][r] * nl2e)) : 0.0f;
+        const float s1 = on ? rcp(1.0f + ex2(v[3][r] * nl2e)) : 0.0f;
+        const float s2 = on && g.m2[r] != 0.0f ? rcp(1.0f + ex2(v[4][r] * nl2e)) : 0.0f;
         const float iS = rcp(fmaxf((s0 + s1) + s2, 1e-6f));
         W.w0[r] = s0 * iS;
         W.w1[r] = s1 * iS;

@@ -1,6 +1,6 @@
-// General Prop2D forward for shapes the paired kernel does not take (lines
-// longer than 256 positions, lines of one position, or bf16 rows of odd
-// width, whose rows are not 4-byte aligned).  A CTA of four warps owns a
+// General Prop2D forward for shapes the direction and sweep-pair kernels do
+// not take (lines longer than 256 positions, lines of one position, or bf16
+// rows of odd width, whose rows are not 4-byte aligned).  A CTA of four warps owns a
 // plane band, warp d runs direction d; each warp keeps its
 // previous and current hidden line in shared memory, lanes stride over the
 // positions of a line, and inputs are read straight from global memory.
@@ -16,7 +16,9 @@ constexpr int kGenericThreads = 128;   // 4 warps: one per direction
 struct GenericParams {
     const void *x, *lam, *wl, *u;
     void *out;
-    int B, Cc, H, W, dirs, share_w;
+    int B, Cc, H, W, dirs;
+    int gate_dirs;          // direction slots of lambda and u: 4, or 1 shared by all directions
+    int w_groups, w_cpg;    // logit fields per (batch, direction) and channels per field
     int n_items, bands, band_rows;
     int hline;      // floats reserved per hidden line (>= max(H, W))
     int y_pitch;
@@ -40,7 +42,6 @@ prop2d_generic_kernel(const GenericParams p) {
     const T *LA = static_cast<const T *>(p.lam);
     const T *U = static_cast<const T *>(p.u);
     const T *WL = static_cast<const T *>(p.wl);
-    const int Cw = p.share_w ? 1 : p.Cc;
 
     for (int e = threadIdx.x; e < p.band_rows * YP; e += kGenericThreads) ys[e] = 0.0f;
     __syncthreads();
@@ -51,8 +52,9 @@ prop2d_generic_kernel(const GenericParams p) {
         const int b = plane / p.Cc, c = plane - b * p.Cc;
         if (active) {
             const size_t xo = (static_cast<size_t>(b) * p.Cc + c) * HW;
-            const size_t go = ((static_cast<size_t>(b) * 4 + d) * p.Cc + c) * HW;
-            const size_t wo = (((static_cast<size_t>(b) * 4 + d) * Cw + (p.share_w ? 0 : c)) * 3) * HW;
+            const size_t go =
+                ((static_cast<size_t>(b) * p.gate_dirs + (p.gate_dirs == 4 ? d : 0)) * p.Cc + c) * HW;
+            const size_t wo = (((static_cast<size_t>(b) * 4 + d) * p.w_groups + c / p.w_cpg) * 3) * HW;
             float *hprev = hbuf, *hcur = hbuf + p.hline;
             for (int q = lane; q < M; q += 32) hprev[q] = 0.0f;
             __syncwarp();

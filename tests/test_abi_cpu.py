@@ -71,7 +71,7 @@ def test_argument_checks(lib, args, status):
 def test_status_strings(lib):
     lib.gspn_status_str.argtypes = [ctypes.c_int]
     lib.gspn_status_str.restype = ctypes.c_char_p
-    for s in range(9):
+    for s in range(11):
         assert lib.gspn_status_str(s).decode().startswith("GSPN_")
     assert lib.gspn_status_str(99) is not None
 
@@ -114,3 +114,22 @@ def test_workspace_ignored_without_share_w(lib):
     assert _fwd_ws(lib)(None, P, P, P, 2, 4, 8, 8, 15, 0, 0, P, None, 0, None) == 1
     assert _fwd_ws(lib)(P, P, P, P, 2, 4, 8, 8, 16, 0, 0, P, None, 0, None) == 3
     assert _fwd_ws(lib)(None, None, None, None, 0, 4, 8, 8, 15, 1, 0, None, None, 0, None) == 0
+
+
+def _fwd_ex(lib):
+    f = lib.gspn_prop2d_fwd_ex
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 8 + [ctypes.c_void_p] * 2
+    f.restype = ctypes.c_int
+    return f
+
+
+@pytest.mark.parametrize("args,status", [
+    ((P, P, P, P, 1, 4, 8, 8, 15, 2, 4, 0, P), 10),       # gate_dirs neither 1 nor 4
+    ((P, P, P, P, 1, 4, 8, 8, 15, 4, 3, 0, P), 10),       # w_groups does not divide Cc
+    ((P, P, P, P, 1, 4, 8, 8, 15, 4, 0, 0, P), 10),       # no logit field
+    ((P, P, P, P, 1, 4, 8, 8, 0, 4, 4, 0, P), 3),         # empty direction mask
+    ((P, P, P, P, -1, 4, 8, 8, 15, 1, 2, 0, P), 2),       # negative B
+    ((None, None, None, None, 0, 4, 8, 8, 15, 1, 2, 0, None), 0),   # empty batch
+])
+def test_ex_argument_checks(lib, args, status):
+    assert _fwd_ex(lib)(*args, None) == status

@@ -82,9 +82,25 @@ def test_reference_arm_other_ranks_are_silent(capsys, monkeypatch):
 def test_profile_traffic_needs_current_sources(tmp_path, monkeypatch, matches):
     os.makedirs(tmp_path / "profiles")
     sha = bench.kernel_sources_sha() if matches else "0" * 64
-    (tmp_path / "profiles" / "prop2d_dir_1k.md").write_text(
+    (tmp_path / "profiles" / "prop2d_pair_1k.md").write_text(
         f"kernel_sources_sha256: {sha}\ntraffic_bytes_per_launch: 12345\n")
     real_sha = bench.kernel_sources_sha()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_sources_sha", lambda: real_sha)
-    assert bench.profiled_traffic("1k") == (12345 if matches else None)
+    assert bench.profiled_traffic("prop2d_pair_kernel", "1k") == (12345 if matches else None)
+    assert bench.profiled_traffic("prop2d_dir_kernel", "1k") is None
+
+
+def test_clock_summary_is_honest_about_short_windows():
+    """A timed region with no clock sample reports the load window, labelled."""
+    cs = bench.ClockSampler(0)
+    cs.proc = object()
+    row = "0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    cs.samples = [(10.0, row), (10.5, row), (11.2, row)]
+    cs.l0, cs.l1, cs.t0, cs.t1 = 9.9, 11.0, 11.05, 11.06
+    out = cs.summary()
+    assert out["timed_region_samples"] == 0 and out["samples"] == 2
+    assert out["source"].startswith("no sample in the timed region")
+    cs.t1 = 11.3
+    out = cs.summary()
+    assert out["source"] == "timed region" and out["samples"] == 1 and out["sm_mhz"] == 1965.0

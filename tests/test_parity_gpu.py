@@ -46,19 +46,41 @@ def oracle_planes(inp, planes, dirs, share_w):
     return np.stack(out)
 
 
+def oracle_all(inp, dirs, share_w):
+    """Oracle output of every plane, computed in (batch, channel-chunk) slices
+    so that the fp64 copies stay small."""
+    B, Cc, H, W = inp["x"].shape
+    chunk = max(1, (1 << 20) // (H * W))
+    out = np.empty(tuple(inp["x"].shape), dtype=np.float64)
+    for b in range(B):
+        for c0 in range(0, Cc, chunk):
+            c1 = min(Cc, c0 + chunk)
+            wl = inp["wlogit"][b:b + 1] if share_w else inp["wlogit"][b:b + 1, :, c0:c1]
+            out[b:b + 1, c0:c1] = oracle.prop2d(
+                f64(inp["x"][b:b + 1, c0:c1]), f64(inp["lam"][b:b + 1, :, c0:c1]), f64(wl),
+                f64(inp["u"][b:b + 1, :, c0:c1]), dirs=dirs, share_w=share_w)
+    return out
+
+
 def workspace(gspn, inp, dirs=15, share_w=1):
     B, Cc, H, W = inp["x"].shape
     n = gspn.workspace_bytes(B, Cc, H, W, dirs, share_w, inp["x"].dtype)
     return torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
 
 
-def check(gspn, inp, dirs=15, share_w=0, planes=None, what="", ws=False):
+def check(gspn, inp, dirs=15, share_w=0, planes=None, what="", ws=False, path=None):
+    """Run the library and compare with the oracle; `path`, when given, is the
+    launch path the call must have taken (gspn_last_launch_info)."""
     d = to_dev(inp)
     kw = {"workspace": workspace(gspn, inp, dirs, share_w)} if ws else {}
     y = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=dirs, share_w=share_w, **kw)
     torch.cuda.synchronize()
+    if path is not None:
+        assert gspn.launch_info()["path"] == path, (what, gspn.launch_info())
     yg = f64(y)
-    if planes is None:
+    if planes == "all":
+        yo = oracle_all(inp, dirs, share_w)
+    elif planes is None:
         yo = oracle.prop2d(f64(inp["x"]), f64(inp["lam"]), f64(inp["wlogit"]), f64(inp["u"]),
                            dirs=dirs, share_w=share_w)
     else:
@@ -83,18 +105,16 @@ def test_workload_full(gspn, name):
     print(f"\n{name}: max|err| / max|y| = {rel:.3e}")
 
 
-@pytest.mark.parametrize("name", ["1k", "2k", "orig"])
-def test_workload_sampled_planes(gspn, name):
-    """Full-size workload in the launch the benchmark times; the oracle checks
-    sampled planes one by one (first, last, and random ones)."""
+@pytest.mark.parametrize("name,path", [("1k", "pair"), ("2k", "dir-shared"),
+                                       ("orig", "dir-yglobal")])
+def test_workload_all_planes(gspn, name, path):
+    """Full-size workload in the launch the benchmark times, every plane
+    compared with the oracle (every item of every persistent CTA, the last
+    partial round included)."""
     w = WORKLOADS[name]
     inp = workload_inputs(w, seed=0)
-    rng = np.random.default_rng(0)
-    n = 3 if name == "orig" else 8
-    planes = [(0, 0), (w.B - 1, w.Cc - 1)]
-    planes += [(int(rng.integers(w.B)), int(rng.integers(w.Cc))) for _ in range(n)]
-    rel = check(gspn, inp, share_w=w.share_w, planes=planes, what=name)
-    print(f"\n{name} (sampled planes): max|err| / max|y| = {rel:.3e}")
+    rel = check(gspn, inp, share_w=w.share_w, planes="all", what=name, path=path)
+    print(f"\n{name} (all planes): max|err| / max|y| = {rel:.3e}")
 
 
 # --------------------------------------------------------------------------
@@ -106,6 +126,10 @@ SHAPES = [
     (2, 2, 33, 31), (1, 3, 32, 32), (1, 2, 64, 65), (2, 2, 74, 74), (1, 2, 16, 100),
     (1, 1, 100, 16), (1, 2, 97, 129), (1, 1, 129, 97), (1, 1, 148, 148), (1, 1, 256, 256),
     (1, 1, 255, 3), (1, 1, 3, 255),
+    # every lane layout of the sweep-pair kernel, odd line counts (the two
+    # sweeps meet on the middle line), non-square grids
+    (2, 2, 2, 2), (2, 3, 5, 6), (1, 2, 37, 38), (1, 2, 38, 36), (1, 2, 50, 50), (1, 2, 81, 82),
+    (1, 2, 112, 112), (1, 2, 128, 128), (1, 2, 40, 64), (1, 2, 96, 80), (3, 5, 74, 74),
 ]
 
 
@@ -138,14 +162,11 @@ def test_share_w(gspn, shape, dtype):
 # --------------------------------------------------------------------------
 
 def test_workload_2k_workspace(gspn):
-    """The 2k compact workload through gspn_prop2d_fwd_ws (sampled planes)."""
+    """The 2k compact workload through gspn_prop2d_fwd_ws (every plane)."""
     w = WORKLOADS["2k"]
     inp = workload_inputs(w, seed=0)
-    rng = np.random.default_rng(1)
-    planes = [(0, 0), (w.B - 1, w.Cc - 1)] + [(int(rng.integers(w.B)), int(rng.integers(w.Cc)))
-                                              for _ in range(8)]
-    rel = check(gspn, inp, share_w=1, planes=planes, what="2k ws", ws=True)
-    print(f"\n2k with workspace (sampled planes): max|err| / max|y| = {rel:.3e}")
+    rel = check(gspn, inp, share_w=1, planes="all", what="2k ws", ws=True, path="dir-shared")
+    print(f"\n2k with workspace (all planes): max|err| / max|y| = {rel:.3e}")
     assert gspn.launch_info()["launches"] == 2
 
 
@@ -167,12 +188,13 @@ def test_share_w_workspace_masks(gspn, dirs, dtype):
     check(gspn, inp, dirs=dirs, share_w=1, what=f"ws dirs={dirs}", ws=True)
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype,W", [("f32", 23), ("bf16", 24)])
 @pytest.mark.parametrize("mode", ["clamp_binds", "all_very_negative", "saturated_positive"])
-def test_share_w_workspace_extremes(gspn, mode, dtype):
+def test_share_w_workspace_extremes(gspn, mode, dtype, W):
     """The clamp (sum of the weights below 1) and saturated logits through the
-    weights normalised ahead."""
-    inp = make_inputs(2, 3, 19, 23, share_w=1, sigma_w=1.0, dtype="f32", seed=3)
+    weights normalised ahead (fp16 weights for bf16 inputs), on the direction
+    kernel that reads them (even width for bf16)."""
+    inp = make_inputs(2, 3, 19, W, share_w=1, sigma_w=1.0, dtype="f32", seed=3)
     g = torch.Generator().manual_seed(6)
     shape = inp["wlogit"].shape
     if mode == "clamp_binds":
@@ -184,7 +206,9 @@ def test_share_w_workspace_extremes(gspn, mode, dtype):
     inp["wlogit"] = wl
     td = torch.bfloat16 if dtype == "bf16" else torch.float32
     inp = {k: v.to(td) for k, v in inp.items()}
-    check(gspn, inp, share_w=1, what=f"ws {mode} {dtype}", ws=True)
+    check(gspn, inp, share_w=1, what=f"ws {mode} {dtype}", ws=True,
+          path="dir-shared" if dtype == "bf16" else "dir")
+    assert gspn.launch_info()["launches"] == 2
 
 
 def test_workspace_unused_without_share_w(gspn):
@@ -211,14 +235,19 @@ def test_hand_examples(gspn, dtype):
         check(gspn, inp, dirs=ex["dirs"][0], what=ex["name"])
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype,shape,path", [
+    ("f32", (1, 2, 19, 23), "pair"), ("bf16", (1, 2, 19, 24), "pair"),
+    ("bf16", (1, 2, 74, 74), "pair"), ("f32", (1, 2, 19, 150), "dir"),
+    ("bf16", (1, 2, 19, 150), "dir-shared"), ("bf16", (1, 2, 19, 23), "generic")],
+    ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 @pytest.mark.parametrize("mode", ["all_very_negative", "clamp_binds", "overflow_pairs",
                                   "saturated_positive", "mixed_extremes"])
-def test_extreme_logits(gspn, mode, dtype):
+def test_extreme_logits(gspn, mode, dtype, shape, path):
     """Logit ranges where the denominator clamp binds (all on-grid logits
     below about -14) or where a product form of the normalisation would
-    overflow (two logits below about -44)."""
-    B, Cc, H, W = 1, 2, 19, 23
+    overflow (two logits below about -44), on each kernel that normalises in
+    the scan (the launch path is asserted)."""
+    B, Cc, H, W = shape
     inp = make_inputs(B, Cc, H, W, sigma_w=1.0, dtype="f32", seed=3)
     g = torch.Generator().manual_seed(5)
     wl = inp["wlogit"]
@@ -239,7 +268,29 @@ def test_extreme_logits(gspn, mode, dtype):
     inp["wlogit"] = wl
     td = torch.bfloat16 if dtype == "bf16" else torch.float32
     inp = {k: v.to(td) for k, v in inp.items()}
-    check(gspn, inp, what=f"{mode} {dtype}")
+    check(gspn, inp, what=f"{mode} {dtype} {shape}", path=path)
+
+
+@pytest.mark.parametrize("dtype,shape,path", [
+    ("f32", (1, 2, 19, 23), "pair"), ("bf16", (2, 3, 74, 74), "pair"),
+    ("f32", (1, 2, 37, 38), "pair"), ("f32", (1, 2, 19, 150), "dir"),
+    ("bf16", (1, 2, 148, 148), "dir-shared"), ("f32", (1, 1, 256, 256), "dir-yglobal"),
+    ("bf16", (1, 2, 19, 23), "generic")],
+    ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
+    """Off-grid logit slots (slot 0 of a line's first position, slot 2 of its
+    last) carry no weight and are never needed; filled with NaN they must not
+    reach the output (the oracle never reads them)."""
+    B, Cc, H, W = shape
+    inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=13)
+    wl = inp["wlogit"].clone()
+    nan = float("nan")
+    wl[:, 0:2, :, 0, :, 0] = nan          # row lines: left end, slot 0
+    wl[:, 0:2, :, 2, :, W - 1] = nan      # row lines: right end, slot 2
+    wl[:, 2:4, :, 0, 0, :] = nan          # column lines: top end, slot 0
+    wl[:, 2:4, :, 2, H - 1, :] = nan      # column lines: bottom end, slot 2
+    inp["wlogit"] = wl
+    check(gspn, inp, what=f"NaN edge slots {shape} {dtype}", path=path)
 
 
 # --------------------------------------------------------------------------
@@ -247,8 +298,12 @@ def test_extreme_logits(gspn, mode, dtype):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "dir-shared"),
-    ((2, 3, 74, 74), "f32", "dir"),
+    ((2, 3, 74, 74), "bf16", "pair"),
+    ((2, 3, 74, 74), "f32", "pair"),
+    ((4, 4, 37, 37), "f32", "pair"),
+    ((1, 4, 16, 16), "f32", "pair"),
+    ((1, 2, 16, 100), "bf16", "pair"),         # short columns in the long rows' layout
+    ((1, 2, 100, 16), "f32", "dir"),           # rows shorter than the pair blocks
     ((1, 2, 160, 160), "f32", "dir-shared"),   # two output planes do not fit
     ((1, 2, 256, 256), "f32", "dir-yglobal"),
     ((1, 2, 256, 256), "bf16", "dir-banded"),
@@ -306,3 +361,34 @@ def test_output_fully_overwritten(gspn):
     gspn.prop2d_fwd(inp["x"], inp["lam"], inp["wlogit"], inp["u"], out=out)
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
+
+
+# --------------------------------------------------------------------------
+# sharing variants: lambda/u shared by the directions, logits by channel groups
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,shape,path", [
+    ("bf16", (2, 4, 74, 74), "pair"), ("f32", (1, 6, 37, 37), "pair"),
+    ("f32", (1, 4, 19, 150), "dir"), ("bf16", (1, 4, 19, 150), "dir-shared"),
+    ("bf16", (1, 4, 20, 33), "generic")],
+    ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+@pytest.mark.parametrize("gate_dirs,groups", [(1, "all"), (4, "half"), (1, "one"), (4, "one")])
+def test_sharing_variants(gspn, dtype, shape, path, gate_dirs, groups):
+    B, Cc, H, W = shape
+    G = {"all": Cc, "half": Cc // 2, "one": 1}[groups]
+    g = torch.Generator().manual_seed(41)
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x = torch.randn((B, Cc, H, W), generator=g)
+    lam = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
+    wl = torch.randn((B, 4, G, 3, H, W), generator=g) * 2.0
+    u = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
+    inp = {k: v.to(td) for k, v in {"x": x, "lam": lam, "wlogit": wl, "u": u}.items()}
+    d = to_dev(inp)
+    y = gspn.prop2d_fwd_ex(d["x"], d["lam"], d["wlogit"], d["u"], gate_dirs=gate_dirs, w_groups=G)
+    torch.cuda.synchronize()
+    assert gspn.launch_info()["path"] == path
+    yo = oracle.prop2d_ex(f64(inp["x"]), f64(inp["lam"]), f64(inp["wlogit"]), f64(inp["u"]),
+                          gate_dirs=gate_dirs, w_groups=G)
+    scale = float(np.max(np.abs(yo)))
+    err = float(np.max(np.abs(f64(y) - yo)))
+    assert err <= TOL[td] * scale, f"{err:.3e} vs {scale:.3e}"
