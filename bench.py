@@ -47,12 +47,15 @@ def peaks():
 
 
 def kernel_sources_sha() -> str:
-    """sha256 over the CUDA sources and the C-ABI header (sorted by name)."""
+    """sha256 over the device-side CUDA sources (sorted by name): every file
+    under csrc/ except gspn_api.cu, the host C ABI (argument checks, planner).
+    The planner's choice is checked separately: a profile also records the
+    launch geometry it was taken with."""
     import glob
     import hashlib
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "spatial_propagation_vision_b200", "csrc", "*")) +
-                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    files = sorted(f for f in glob.glob(os.path.join(ROOT, "spatial_propagation_vision_b200", "csrc", "*"))
+                   if os.path.basename(f) != "gspn_api.cu")
     for f in files:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
@@ -69,9 +72,10 @@ def profile_path(kernel: str, workload: str) -> str:
     return os.path.join(ROOT, "profiles", f"{kernel.replace('_kernel', '')}_{workload}.md")
 
 
-def profiled_traffic(kernel: str, workload: str):
+def profiled_traffic(kernel: str, workload: str, launch: dict | None = None):
     """DRAM bytes per launch from the committed ncu summary of this kernel on
-    this workload, if it was captured on the current kernel sources; else None."""
+    this workload, if it was captured on the current device sources and (when
+    `launch` is given) with the same grid, block and shared memory; else None."""
     import re
     path = profile_path(kernel, workload)
     if not os.path.exists(path):
@@ -81,6 +85,10 @@ def profiled_traffic(kernel: str, workload: str):
     tb = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
     if not sha or not tb or sha.group(1) != kernel_sources_sha():
         return None
+    if launch is not None:
+        geo = re.search(r"launch_geometry:\s*grid=(\d+)\s+block=(\d+)\s+smem=(\d+)", text)
+        if not geo or tuple(int(g) for g in geo.groups()) != (launch["grid"], launch["block"], launch["smem"]):
+            return None
     return int(tb.group(1))
 
 
@@ -408,7 +416,7 @@ def run_ours(args, w):
     peak, peak_kind = peaks()
     achieved = nbytes / (avg_kernel_ms * 1e-3) / 1e9
     kernel = KERNEL_OF_PATH.get(info["path"], info["path"])
-    traffic = args.traffic if args.traffic is not None else profiled_traffic(kernel, w.name)
+    traffic = args.traffic if args.traffic is not None else profiled_traffic(kernel, w.name, info)
     value = job_value(nbytes, world, step_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -450,6 +458,9 @@ def main():
     ap.add_argument("--ref-planes", type=int, default=64, help="oracle planes per reference step")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--cc", type=int, default=None,
+                    help="override the workload's channel count (a smaller case of the same "
+                         "kernel, for ncu captures that must stay within a few GB)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if captured for "
                          "the current build")
@@ -457,6 +468,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.cc is not None:
+        import dataclasses
+        w = dataclasses.replace(w, Cc=args.cc, name=f"{w.name}-cc{args.cc}")
     if args.impl == "reference":
         run_reference(args, w)
     else:

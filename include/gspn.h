@@ -233,6 +233,35 @@ gspn_status gspn_prop2d_fwd_noalloc(const void *x, const void *lambda, const voi
                                     int share_w, gspn_dtype dtype, void *out,
                                     cudaStream_t stream);
 
+/*
+ * gspn_prop2d_bwd -- gradients of y = Prop2D(x; u, lambda, w) (the pages
+ * report the backward kernel's speed-ups, Sec. 6.1 "Scaling with input size,
+ * batch, and channels", Fig. 8; the gradients are the chain rule of the
+ * forward recurrence and normalisation).
+ *
+ * Given gy = dL/dy ([B][Cc][H][W], dtype `dtype`), writes fp32 gradients in
+ * the input layouts:
+ *   dx       [B][Cc][H][W]          sum over the enabled directions
+ *   dlambda  [B][4][Cc][H][W]       0 in slots of directions not enabled
+ *   dwlogit  [B][4][Cw][3][H][W]    through sigmoid, local sum, clamp and
+ *                                   divide; 0 in off-grid slots; with
+ *                                   share_w = 1 summed over the channels
+ *   du       [B][4][Cc][H][W]
+ * The clamp of the local sum is differentiated on the branch the forward
+ * takes (sum above 1e-6: the sum; else the constant 1e-6).
+ *
+ * x, lambda, wlogit, u, gy : device pointers, dtype `dtype`, read only.
+ * dx, dlambda, dwlogit, du : device fp32 buffers; zeroed on `stream` by the
+ *                            call and then written.
+ * Lines (H, W) up to 256.  All pointers 16-byte aligned.  Asynchronous on
+ * `stream`; one kernel launch after four cudaMemsetAsync.  Other arguments
+ * and errors as gspn_prop2d_fwd.
+ */
+gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const void *wlogit,
+                            const void *u, const void *gy, int B, int Cc, int H, int W, int dirs,
+                            int share_w, gspn_dtype dtype, float *dx, float *dlambda,
+                            float *dwlogit, float *du, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gspn_status_str(gspn_status status);
 

@@ -215,6 +215,13 @@ cudaError_t try_pair(const void *x, const void *lambda, const void *wlogit, cons
     taken = false;
     const int mx = H > W ? H : W;
     if (H < 2 || W < 2 || mx > kMaxPairLine || (es == 2 && W % 2)) return cudaSuccess;
+    // Measured on B200 against the direction kernel: the sweep-pair kernel is
+    // faster for lines of up to 16 positions (16 x 16, fp32: 0.0156 vs
+    // 0.0174 ms) and for the row directions alone (74 x 74, bf16: 0.229 vs
+    // 0.253 ms), slower when column directions take part on longer lines
+    // (74 x 74, bf16, four directions: 0.52 vs 0.33 ms; its one column warp
+    // per plane runs both column sweeps).  It takes the shapes where it wins.
+    if (mx > 16 && (dirs & 12) != 0) return cudaSuccess;
     const int bucket = (mx + 15) / 16 - 1;           // 0 .. 7
     const int RP = bucket / 2, NS = bucket % 2 + 1;  // capacity 32 RP + 16 NS >= mx
     if (W < 32 * RP) return cudaSuccess;
@@ -475,4 +482,54 @@ extern "C" gspn_status gspn_prop2d_fwd_noalloc(const void *x, const void *lambda
     if (need > 0 && noalloc_scratch(&ws) != cudaSuccess) return GSPN_ERR_CUDA;
     return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{4, share_w ? 1 : Cc}, dtype,
                       out, ws, stream);
+}
+
+// ---------------------------------------------------------------------------
+// gspn_prop2d_bwd: gradients of Prop2D
+// ---------------------------------------------------------------------------
+
+namespace {
+constexpr int kMaxBwdLine = 256;   // lines the backward kernel holds (8 positions per lane)
+}  // namespace
+
+extern "C" gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const void *wlogit,
+                                       const void *u, const void *gy, int B, int Cc, int H, int W,
+                                       int dirs, int share_w, gspn_dtype dtype, float *dx,
+                                       float *dlambda, float *dwlogit, float *du,
+                                       cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
+    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
+    if (dtype != GSPN_F32 && dtype != GSPN_BF16) return GSPN_ERR_DTYPE;
+    if (B == 0 || Cc == 0 || H == 0 || W == 0) return GSPN_OK;
+    if (!x || !lambda || !wlogit || !u || !gy || !dx || !dlambda || !dwlogit || !du)
+        return GSPN_ERR_NULL;
+    if (misaligned(x) || misaligned(lambda) || misaligned(wlogit) || misaligned(u) || misaligned(gy) ||
+        misaligned(dx) || misaligned(dlambda) || misaligned(dwlogit) || misaligned(du))
+        return GSPN_ERR_ALIGN;
+    const int maxline = H > W ? H : W;
+    if (maxline > kMaxBwdLine || static_cast<long long>(H) * W > (1LL << 30) ||
+        static_cast<long long>(B) * Cc > 0x7fffffffLL)
+        return GSPN_ERR_SHAPE;
+    DeviceProps dp;
+    if (device_props(dp) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (dp.major != 10) return GSPN_ERR_DEVICE;
+    const size_t plane = static_cast<size_t>(H) * W * sizeof(float);
+    const size_t nx = static_cast<size_t>(B) * Cc * plane;
+    const size_t nw = static_cast<size_t>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane;
+    if (cudaMemsetAsync(dx, 0, nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemsetAsync(dlambda, 0, 4 * nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemsetAsync(du, 0, 4 * nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemsetAsync(dwlogit, 0, nw, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    gspn::BwdParams bp{};
+    bp.x = x; bp.lam = lambda; bp.wl = wlogit; bp.u = u; bp.gy = gy;
+    bp.dx = dx; bp.dlam = dlambda; bp.dwl = dwlogit; bp.du = du;
+    bp.B = B; bp.Cc = Cc; bp.H = H; bp.W = W; bp.dirs = dirs; bp.share_w = share_w;
+    bp.R = (maxline + 31) / 32;
+    bp.n_ckpt = (maxline + gspn::kBwdSeg - 1) / gspn::kBwdSeg;
+    bp.warp_floats = (bp.n_ckpt + gspn::kBwdSeg + 1) * 32 * bp.R;
+    const int smem = 4 * bp.warp_floats * static_cast<int>(sizeof(float));
+    if (smem > dp.smem_optin) return GSPN_ERR_SHAPE;
+    const cudaError_t e = launch_bwd(bp, dtype == GSPN_BF16, smem, dp, stream, g_last);
+    return e == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
 }

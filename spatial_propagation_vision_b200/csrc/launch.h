@@ -11,6 +11,7 @@
 #include "prop2d_generic.cuh"
 #include "prop2d_norm.cuh"
 #include "prop2d_pair.cuh"
+#include "prop2d_bwd.cuh"
 
 namespace gspn_host {
 
@@ -57,6 +58,10 @@ cudaError_t launch_pair_f32(int RP, int NS, const gspn::PairParams &pp, int smem
 // memory; sets the kernel's shared-memory limit.  Both are cached per
 // (device, kernel, smem), so repeated calls make no runtime queries.
 cudaError_t kernel_occupancy(const void *kernel, int threads, int smem, int &per_sm);
+
+// Backward kernel (fp32 gradients); the caller zeroed the gradient buffers.
+cudaError_t launch_bwd(const gspn::BwdParams &bp, bool bf16, int smem, const DeviceProps &dp,
+                       cudaStream_t s, LaunchInfo &li);
 
 // Normalised weights of the compact mode into the workspace (one launch).
 cudaError_t launch_norm(const gspn::NormParams &np, bool bf16, const DeviceProps &dp, cudaStream_t s);

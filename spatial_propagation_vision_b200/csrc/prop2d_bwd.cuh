@@ -1,0 +1,248 @@
+// Backward of Prop2D: the vector-Jacobian product of the forward recurrence
+// and normalisation ("Scaling Parallel Sequence Models to Foundation-Scale
+// Vision Encoders", Sec. 6.1 "Scaling with input size, batch, and channels",
+// Fig. 8 reports the backward kernel's timings; the backward itself is the
+// chain rule of Sec. 3 "Line-scan recurrence" and Sec. 5.1 "Fused CUDA
+// normalization").
+//
+// Given gy = dL/dy, for every (batch, channel, enabled direction):
+//
+//     g_l       = u_l gy_l + W_{l+1}^T g_{l+1}          (adjoint, reverse scan order)
+//     du_l      = gy_l h_l
+//     dlambda_l = g_l x_l,      dx_l += g_l lambda_l
+//     dw_l(q,k) = g_l(q) h_{l-1}(q+k-1)
+//     dz_j      = ds_j s_j (1 - s_j),   ds_j = (dw_j - sum_k dw_k w_k) / S
+//                 (S = sum of the on-grid sigmoids; dw_j / eps when the clamp
+//                 holds the denominator at eps)
+//
+// One CTA of four warps owns one (batch, channel) plane; warp d runs
+// direction d.  Lane l holds positions l*R .. l*R + R - 1 of a line.  The
+// forward lines are recomputed: a first sweep keeps h at every kSeg-th line
+// (checkpoints) in shared memory; the reverse sweep then replays each
+// segment of kSeg lines from its checkpoint into a segment buffer and walks
+// it backwards.  Shared memory per warp: (L / kSeg + kSeg + 1) lines.
+// Weights are recomputed in the plain form (sigmoid, local sum, clamp,
+// divide) in fp32 in both sweeps.  Gradients are fp32: dlambda, du and (per
+// channel) dwlogit are stored once; dx adds the four directions with global
+// fp32 atomics, and shared logit fields (share_w) add over the channels
+// likewise, into buffers the host zeroed.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "device_common.cuh"
+
+namespace gspn {
+
+constexpr int kBwdThreads = 128;   // warp d runs direction d
+constexpr int kBwdSeg = 16;        // lines per recomputed segment
+
+struct BwdParams {
+    const void *x, *lam, *wl, *u, *gy;
+    float *dx, *dlam, *dwl, *du;
+    int B, Cc, H, W, dirs, share_w;
+    int R;            // positions per lane (line capacity 32 R >= max(H, W))
+    int n_ckpt;       // checkpoint lines per warp (ceil(maxL / kBwdSeg))
+    int warp_floats;  // shared-memory floats per warp
+};
+
+template <typename T> __device__ __forceinline__ float bwd_in(const T *p, size_t i);
+template <> __device__ __forceinline__ float bwd_in<float>(const float *p, size_t i) { return __ldg(p + i); }
+template <> __device__ __forceinline__ float bwd_in<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+
+// sigmoid in fp32 (hardware 2^x and reciprocal), saturating to 0 or 1
+__device__ __forceinline__ float bwd_sigmoid(float z) {
+    return rcp(1.0f + ex2(z * -1.4426950408889634f));
+}
+
+template <typename T, int R>
+struct BwdLine {
+    const BwdParams &p;
+    const int lane, d;
+    const bool fwd, rows;
+    const int L, M;
+    const T *x, *lam, *u, *gy, *wl;   // this plane's tensors (direction d)
+    float *dx, *dlam, *du, *dwl;
+
+    __device__ BwdLine(const BwdParams &p_, int lane_, int d_, int b, int c)
+        : p(p_), lane(lane_), d(d_), fwd((d_ & 1) == 0), rows(d_ < 2),
+          L(d_ < 2 ? p_.H : p_.W), M(d_ < 2 ? p_.W : p_.H) {
+        const size_t HW = static_cast<size_t>(p.H) * p.W;
+        const size_t xo = (static_cast<size_t>(b) * p.Cc + c) * HW;
+        const size_t go = ((static_cast<size_t>(b) * 4 + d) * p.Cc + c) * HW;
+        const int Cw = p.share_w ? 1 : p.Cc;
+        const size_t wo = (((static_cast<size_t>(b) * 4 + d) * Cw + (p.share_w ? 0 : c)) * 3) * HW;
+        x = static_cast<const T *>(p.x) + xo;
+        gy = static_cast<const T *>(p.gy) + xo;
+        lam = static_cast<const T *>(p.lam) + go;
+        u = static_cast<const T *>(p.u) + go;
+        wl = static_cast<const T *>(p.wl) + wo;
+        dx = p.dx + xo;
+        dlam = p.dlam + go;
+        du = p.du + go;
+        dwl = p.dwl + wo;
+    }
+
+    // element index of position q of scan step s within a plane
+    __device__ __forceinline__ size_t idx(int s, int q) const {
+        const int line = fwd ? s : L - 1 - s;
+        return rows ? static_cast<size_t>(line) * p.W + q : static_cast<size_t>(q) * p.W + line;
+    }
+
+    // normalised weights (w), sigmoids (s) and local sum (S) of position q
+    __device__ __forceinline__ void weights(size_t e, int q, float (&s)[3], float (&w)[3], float &S) const {
+        const size_t HW = static_cast<size_t>(p.H) * p.W;
+        S = 0.f;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int nb = q + k - 1;
+            s[k] = (nb >= 0 && nb < M) ? bwd_sigmoid(bwd_in(wl, k * HW + e)) : 0.f;
+            S += s[k];
+        }
+        const float r = 1.0f / fmaxf(S, 1e-6f);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) w[k] = s[k] * r;
+    }
+
+    // one forward step: h <- W h + lambda x (positions past the end stay 0)
+    __device__ __forceinline__ void fwd_step(int s, float (&h)[R]) const {
+        const float hl = __shfl_up_sync(0xffffffffu, h[R - 1], 1);
+        const float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
+        float hn[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = lane * R + r;
+            if (q >= M) { hn[r] = 0.f; continue; }
+            const size_t e = idx(s, q);
+            float sg[3], w[3], S;
+            weights(e, q, sg, w, S);
+            const float left = r > 0 ? h[r > 0 ? r - 1 : 0] : (lane > 0 ? hl : 0.f);
+            const float right = r + 1 < R ? h[r + 1 < R ? r + 1 : r] : hr;
+            hn[r] = w[0] * left + w[1] * h[r] + w[2] * right + bwd_in(lam, e) * bwd_in(x, e);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) h[r] = hn[r];
+    }
+
+    __device__ __forceinline__ void store_line(float *buf, const float (&h)[R]) const {
+#pragma unroll
+        for (int r = 0; r < R; ++r) buf[lane * R + r] = h[r];
+    }
+    __device__ __forceinline__ void load_line(const float *buf, float (&h)[R]) const {
+#pragma unroll
+        for (int r = 0; r < R; ++r) h[r] = buf[lane * R + r];
+    }
+
+    // The whole backward of this direction.  `ck`: checkpoint lines
+    // (line i holds h after step i * kSeg + kSeg - 1), `seg`: kSeg + 1 lines
+    // (line 0: h before the segment, line 1 + t: after its step t).
+    __device__ void run(float *ck, float *seg) const {
+        const int line_f = 32 * R;
+        float h[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) h[r] = 0.f;
+        // forward sweep: checkpoints at the end of every segment
+        for (int s = 0; s < L; ++s) {
+            fwd_step(s, h);
+            if (s % kBwdSeg == kBwdSeg - 1) store_line(ck + (s / kBwdSeg) * line_f, h);
+        }
+        __syncwarp();
+        float carry[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) carry[r] = 0.f;
+        const int nseg = (L + kBwdSeg - 1) / kBwdSeg;
+        for (int sg = nseg - 1; sg >= 0; --sg) {
+            const int s0 = sg * kBwdSeg, s1 = min(L, s0 + kBwdSeg);
+            // replay the segment: seg[0] = h before step s0, seg[1 + t] after step s0 + t
+            if (sg == 0) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) h[r] = 0.f;
+            } else {
+                load_line(ck + (sg - 1) * line_f, h);
+            }
+            store_line(seg, h);
+            for (int s = s0; s < s1; ++s) {
+                fwd_step(s, h);
+                store_line(seg + (s - s0 + 1) * line_f, h);
+            }
+            __syncwarp();
+            // reverse steps of the segment
+            for (int s = s1 - 1; s >= s0; --s) {
+                const float *hcur = seg + (s - s0 + 1) * line_f;
+                const float *hprv = seg + (s - s0) * line_f;
+                float adj[R], cl = 0.f, cr = 0.f, cmid[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    adj[r] = 0.f;
+                    cmid[r] = 0.f;
+                }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const int q = lane * R + r;
+                    if (q >= M) continue;
+                    const size_t e = idx(s, q);
+                    const float gyv = bwd_in(gy, e);
+                    const float a = bwd_in(u, e) * gyv + carry[r];
+                    adj[r] = a;
+                    du[e] = gyv * hcur[q];
+                    dlam[e] = a * bwd_in(x, e);
+                    atomicAdd(dx + e, a * bwd_in(lam, e));
+                    float sgm[3], w[3], S;
+                    weights(e, q, sgm, w, S);
+                    float dw[3], dot = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        const int nb = q + k - 1;
+                        dw[k] = (nb >= 0 && nb < M && s > 0) ? a * hprv[nb] : 0.f;
+                        dot += dw[k] * w[k];
+                    }
+                    const size_t HW = static_cast<size_t>(p.H) * p.W;
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        const int nb = q + k - 1;
+                        if (nb < 0 || nb >= M) continue;
+                        const float ds = S > 1e-6f ? (dw[k] - dot) / S : dw[k] * 1e6f;
+                        const float dz = ds * sgm[k] * (1.f - sgm[k]);
+                        if (p.share_w) atomicAdd(dwl + k * HW + e, dz);
+                        else dwl[k * HW + e] = dz;
+                    }
+                    // transposed stencil: position q passes w_k a to q + k - 1
+                    const float c0 = w[0] * a, c1 = w[1] * a, c2 = w[2] * a;
+                    cmid[r] += c1;
+                    if (r > 0) cmid[r - 1 > 0 ? r - 1 : 0] += c0;
+                    else cl = c0;
+                    if (r + 1 < R) cmid[r + 1 < R ? r + 1 : r] += c2;
+                    else cr = c2;
+                }
+                // contributions that cross lanes
+                const float from_right = __shfl_down_sync(0xffffffffu, cl, 1);   // lane+1's position 0 -> my last
+                const float from_left = __shfl_up_sync(0xffffffffu, cr, 1);      // lane-1's last -> my first
+#pragma unroll
+                for (int r = 0; r < R; ++r) carry[r] = cmid[r];
+                if (lane < 31) carry[R - 1] += from_right;
+                if (lane > 0) carry[0] += from_left;
+            }
+            __syncwarp();
+        }
+    }
+};
+
+template <typename T, int R>
+__global__ void __launch_bounds__(kBwdThreads) prop2d_bwd_kernel(const BwdParams p) {
+    extern __shared__ __align__(16) float bsm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (!((p.dirs >> warp) & 1)) return;
+    float *ck = bsm + warp * p.warp_floats;
+    float *seg = ck + p.n_ckpt * 32 * R;
+    for (int plane = blockIdx.x; plane < p.B * p.Cc; plane += gridDim.x) {
+        const int b = plane / p.Cc, c = plane - b * p.Cc;
+        BwdLine<T, R> ln(p, lane, warp, b, c);
+        ln.run(ck, seg);
+        __syncwarp();
+    }
+}
+
+}  // namespace gspn

@@ -38,6 +38,8 @@ lib.gspn_prop2d_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _
 lib.gspn_prop2d_fwd_ws.restype = _i
 lib.gspn_prop2d_fwd_ex.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 8 + [_vp, _vp]
 lib.gspn_prop2d_fwd_ex.restype = _i
+lib.gspn_prop2d_bwd.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 5
+lib.gspn_prop2d_bwd.restype = _i
 lib.gspn_prop2d_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
 lib.gspn_prop2d_fwd_noalloc.restype = _i
 lib.gspn_prop2d_workspace_bytes.argtypes = [_i] * 7
@@ -163,6 +165,38 @@ def prop2d_fwd_ex(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: t
     if st != 0:
         raise GspnError(st)
     return out
+
+
+def prop2d_bwd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torch.Tensor,
+               gy: torch.Tensor, dirs: int = 15, share_w: int = 0,
+               stream: torch.cuda.Stream | None = None) -> dict:
+    """Gradients of Prop2D (gspn_prop2d_bwd) for the upstream gradient gy
+    ([B,Cc,H,W], dtype of x): fp32 tensors {"x", "lam", "wlogit", "u"} in the
+    input layouts."""
+    B, Cc, H, W = _dims(x)
+    if x.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    Cw = 1 if share_w else Cc
+    dev = x.device
+    _check("x", x, (B, Cc, H, W), x.dtype, dev)
+    _check("gy", gy, (B, Cc, H, W), x.dtype, dev)
+    _check("lam", lam, (B, 4, Cc, H, W), x.dtype, dev)
+    _check("u", u, (B, 4, Cc, H, W), x.dtype, dev)
+    _check("wlogit", wlogit, (B, 4, Cw, 3, H, W), x.dtype, dev)
+    g = {"x": torch.empty((B, Cc, H, W), dtype=torch.float32, device=dev),
+         "lam": torch.empty((B, 4, Cc, H, W), dtype=torch.float32, device=dev),
+         "wlogit": torch.empty((B, 4, Cw, 3, H, W), dtype=torch.float32, device=dev),
+         "u": torch.empty((B, 4, Cc, H, W), dtype=torch.float32, device=dev)}
+    with torch.cuda.device(dev):
+        st = lib.gspn_prop2d_bwd(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(), u.data_ptr(),
+                                 gy.data_ptr(), B, Cc, H, W, int(dirs), int(share_w), _DT[x.dtype],
+                                 g["x"].data_ptr(), g["lam"].data_ptr(), g["wlogit"].data_ptr(),
+                                 g["u"].data_ptr(), _stream_handle(stream))
+    if st != 0:
+        raise GspnError(st)
+    return g
 
 
 def prop2d_fwd_noalloc(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor,

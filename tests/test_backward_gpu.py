@@ -1,0 +1,85 @@
+"""GPU parity of the backward (gspn_prop2d_bwd) against the fp64 backward
+oracle, gradient by gradient: max |g_gpu - g_oracle| <= tol * max |g_oracle|
+with tol = 1e-4 for fp32 inputs and 2e-2 for bf16 inputs (the oracle sees the
+same bf16-rounded inputs and upstream gradient)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from spatial_propagation_vision_b200.workloads import WORKLOADS, make_inputs, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+
+@pytest.fixture(scope="module")
+def gspn():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from spatial_propagation_vision_b200 import prop2d
+    return prop2d
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def check_bwd(gspn, inp, dirs=15, share_w=0, seed=0, what=""):
+    g = torch.Generator().manual_seed(seed)
+    gy = torch.randn(inp["x"].shape, generator=g).to(inp["x"].dtype)
+    d = {k: v.cuda() for k, v in inp.items()}
+    got = gspn.prop2d_bwd(d["x"], d["lam"], d["wlogit"], d["u"], gy.cuda(), dirs=dirs,
+                          share_w=share_w)
+    torch.cuda.synchronize()
+    assert gspn.launch_info()["path"] == "bwd"
+    want = oracle.prop2d_bwd(f64(inp["x"]), f64(inp["lam"]), f64(inp["wlogit"]), f64(inp["u"]),
+                             f64(gy), dirs=dirs, share_w=share_w)
+    tol = TOL[inp["x"].dtype]
+    worst = 0.0
+    for k in ("x", "lam", "wlogit", "u"):
+        a, b = f64(got[k]), want[k]
+        assert np.all(np.isfinite(a)), f"{what}: d{k} not finite"
+        scale = float(np.max(np.abs(b)))
+        err = float(np.max(np.abs(a - b)))
+        assert err <= tol * max(scale, 1e-30), f"{what}: d{k} err {err:.3e} > {tol} * {scale:.3e}"
+        worst = max(worst, err / max(scale, 1e-30))
+    return worst
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1), (1, 2, 5, 7), (2, 3, 16, 16), (1, 2, 37, 38),
+                                   (1, 2, 33, 17), (2, 2, 74, 74), (1, 1, 100, 130),
+                                   (1, 1, 256, 256)], ids=lambda s: "x".join(map(str, s)))
+def test_backward_shapes(gspn, shape, dtype):
+    B, Cc, H, W = shape
+    inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=sum(shape))
+    check_bwd(gspn, inp, seed=1, what=f"{shape} {dtype}")
+
+
+@pytest.mark.parametrize("dirs", [1, 2, 4, 8, 5, 10, 3, 12])
+def test_backward_direction_masks(gspn, dirs):
+    inp = make_inputs(1, 2, 19, 22, sigma_w=2.0, dtype="f32", seed=dirs)
+    check_bwd(gspn, inp, dirs=dirs, seed=2, what=f"dirs={dirs}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_share_w(gspn, dtype):
+    inp = make_inputs(2, 3, 19, 24, share_w=1, sigma_w=1.5, dtype=dtype, seed=5)
+    check_bwd(gspn, inp, share_w=1, seed=3, what=f"share_w {dtype}")
+
+
+def test_backward_clamped(gspn):
+    """Logits near -15: the clamp holds the local sum's denominator."""
+    inp = make_inputs(1, 2, 9, 10, sigma_w=1.0, dtype="f32", seed=6)
+    g = torch.Generator().manual_seed(7)
+    inp["wlogit"] = -15.0 + 0.05 * (2 * torch.rand(inp["wlogit"].shape, generator=g) - 1)
+    check_bwd(gspn, inp, seed=4, what="clamped")
+
+
+def test_backward_1k_workload(gspn):
+    """The 1k workload's shape (B=32, Cc=64, 74x74, bf16), every plane."""
+    w = WORKLOADS["1k"]
+    rel = check_bwd(gspn, workload_inputs(w, seed=0), seed=9, what="1k")
+    print(f"\n1k backward: worst max|err| / max|g| = {rel:.3e}")

@@ -83,12 +83,17 @@ def test_profile_traffic_needs_current_sources(tmp_path, monkeypatch, matches):
     os.makedirs(tmp_path / "profiles")
     sha = bench.kernel_sources_sha() if matches else "0" * 64
     (tmp_path / "profiles" / "prop2d_pair_1k.md").write_text(
-        f"kernel_sources_sha256: {sha}\ntraffic_bytes_per_launch: 12345\n")
+        f"kernel_sources_sha256: {sha}\ntraffic_bytes_per_launch: 12345\n"
+        "launch_geometry: grid=444 block=128 smem=53552\n")
     real_sha = bench.kernel_sources_sha()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_sources_sha", lambda: real_sha)
     assert bench.profiled_traffic("prop2d_pair_kernel", "1k") == (12345 if matches else None)
     assert bench.profiled_traffic("prop2d_dir_kernel", "1k") is None
+    same = {"grid": 444, "block": 128, "smem": 53552}
+    other = dict(same, grid=592)
+    assert bench.profiled_traffic("prop2d_pair_kernel", "1k", same) == (12345 if matches else None)
+    assert bench.profiled_traffic("prop2d_pair_kernel", "1k", other) is None
 
 
 def test_clock_summary_is_honest_about_short_windows():

@@ -105,7 +105,7 @@ def test_workload_full(gspn, name):
     print(f"\n{name}: max|err| / max|y| = {rel:.3e}")
 
 
-@pytest.mark.parametrize("name,path", [("1k", "pair"), ("2k", "dir-shared"),
+@pytest.mark.parametrize("name,path", [("1k", "dir-shared"), ("2k", "dir-shared"),
                                        ("orig", "dir-yglobal")])
 def test_workload_all_planes(gspn, name, path):
     """Full-size workload in the launch the benchmark times, every plane
@@ -236,8 +236,9 @@ def test_hand_examples(gspn, dtype):
 
 
 @pytest.mark.parametrize("dtype,shape,path", [
-    ("f32", (1, 2, 19, 23), "pair"), ("bf16", (1, 2, 19, 24), "pair"),
-    ("bf16", (1, 2, 74, 74), "pair"), ("f32", (1, 2, 19, 150), "dir"),
+    ("f32", (1, 2, 19, 23), "dir"), ("bf16", (1, 2, 19, 24), "dir-shared"),
+    ("bf16", (1, 2, 74, 74), "dir-shared"), ("f32", (1, 2, 16, 16), "pair"),
+    ("bf16", (1, 2, 16, 16), "pair"), ("f32", (1, 2, 19, 150), "dir"),
     ("bf16", (1, 2, 19, 150), "dir-shared"), ("bf16", (1, 2, 19, 23), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 @pytest.mark.parametrize("mode", ["all_very_negative", "clamp_binds", "overflow_pairs",
@@ -272,8 +273,8 @@ def test_extreme_logits(gspn, mode, dtype, shape, path):
 
 
 @pytest.mark.parametrize("dtype,shape,path", [
-    ("f32", (1, 2, 19, 23), "pair"), ("bf16", (2, 3, 74, 74), "pair"),
-    ("f32", (1, 2, 37, 38), "pair"), ("f32", (1, 2, 19, 150), "dir"),
+    ("f32", (1, 2, 16, 15), "pair"), ("bf16", (2, 3, 74, 74), "dir-shared"),
+    ("f32", (1, 2, 37, 38), "dir"), ("f32", (1, 2, 19, 150), "dir"),
     ("bf16", (1, 2, 148, 148), "dir-shared"), ("f32", (1, 1, 256, 256), "dir-yglobal"),
     ("bf16", (1, 2, 19, 23), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
@@ -298,11 +299,11 @@ def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "pair"),
-    ((2, 3, 74, 74), "f32", "pair"),
-    ((4, 4, 37, 37), "f32", "pair"),
+    ((2, 3, 74, 74), "bf16", "dir-shared"),
+    ((2, 3, 74, 74), "f32", "dir"),
+    ((4, 4, 37, 37), "f32", "dir"),
     ((1, 4, 16, 16), "f32", "pair"),
-    ((1, 2, 16, 100), "bf16", "pair"),         # short columns in the long rows' layout
+    ((2, 2, 16, 14), "bf16", "pair"),
     ((1, 2, 100, 16), "f32", "dir"),           # rows shorter than the pair blocks
     ((1, 2, 160, 160), "f32", "dir-shared"),   # two output planes do not fit
     ((1, 2, 256, 256), "f32", "dir-yglobal"),
@@ -368,7 +369,7 @@ def test_output_fully_overwritten(gspn):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dtype,shape,path", [
-    ("bf16", (2, 4, 74, 74), "pair"), ("f32", (1, 6, 37, 37), "pair"),
+    ("bf16", (2, 4, 74, 74), "dir-shared"), ("f32", (1, 6, 16, 16), "pair"),
     ("f32", (1, 4, 19, 150), "dir"), ("bf16", (1, 4, 19, 150), "dir-shared"),
     ("bf16", (1, 4, 20, 33), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
@@ -392,3 +393,20 @@ def test_sharing_variants(gspn, dtype, shape, path, gate_dirs, groups):
     scale = float(np.max(np.abs(yo)))
     err = float(np.max(np.abs(f64(y) - yo)))
     assert err <= TOL[td] * scale, f"{err:.3e} vs {scale:.3e}"
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 3, 74, 74), (1, 2, 37, 38), (1, 2, 50, 50), (1, 2, 81, 82),
+                                   (1, 2, 112, 112), (1, 2, 128, 128), (1, 2, 40, 64),
+                                   (1, 2, 96, 80), (1, 2, 16, 100), (3, 5, 21, 18)],
+                         ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("dirs", [1, 2, 3])
+def test_row_directions_on_the_sweep_pair_kernel(gspn, shape, dtype, dirs):
+    """Row directions alone run on the sweep-pair kernel for lines up to 128
+    (every lane layout: pairs plus one or two singles per lane)."""
+    B, Cc, H, W = shape
+    if dtype == "bf16" and W % 2:
+        pytest.skip("odd bf16 rows go to the general kernel")
+    inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=dirs + sum(shape))
+    want = "pair" if W >= 32 * (((max(H, W) + 15) // 16 - 1) // 2) else None
+    check(gspn, inp, dirs=dirs, what=f"rows {shape} {dtype} dirs={dirs}", path=want)
