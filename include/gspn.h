@@ -174,11 +174,16 @@ gspn_status gspn_prop2d_fwd_ws(const void *x, const void *lambda, const void *wl
  * gspn_prop2d_fwd_host -- the same operation on HOST buffers.
  *
  * Copies the four host inputs (h_x, h_lambda, h_wlogit, h_u) into the
- * caller's device buffers (d_x, d_lambda, d_wlogit, d_u) with
- * cudaMemcpyAsync on `stream`, runs gspn_prop2d_fwd into d_out, copies d_out
- * back into h_out, and synchronises `stream` before returning, so h_out is
- * valid on return.  Host buffers should be pinned (page-locked) for the
- * copies to run at full speed; pageable memory works but is slower.  Device
+ * caller's device buffers (d_x, d_lambda, d_wlogit, d_u), runs
+ * gspn_prop2d_fwd into d_out and copies d_out back into h_out, in up to four
+ * batch chunks whose uploads, kernels and downloads overlap (chunk k+1 is
+ * uploaded while chunk k runs and chunk k-1 comes back).  The chunks run on
+ * three streams and a few events that the library creates once per device
+ * (no device memory); they start after the work already queued on `stream`.
+ * Returns after everything has finished, so h_out is valid on return.
+ * Calls from several host threads on one device are serialised.  Host
+ * buffers should be pinned (page-locked) for the copies to run at full
+ * speed and to overlap; pageable memory works but is slower.  Device
  * buffers follow the rules of gspn_prop2d_fwd.  Nothing is allocated.
  */
 gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda, const void *h_wlogit,

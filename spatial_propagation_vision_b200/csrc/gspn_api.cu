@@ -405,6 +405,45 @@ extern "C" gspn_status gspn_prop2d_fwd_ws(const void *x, const void *lambda, con
                       out, need > 0 ? workspace : nullptr, stream);
 }
 
+namespace {
+
+constexpr int kHostChunks = 4;   // batch chunks of the pipelined host entry point
+
+// Streams and events of the host entry point's pipeline, made once per
+// device: uploads, kernels and downloads of consecutive batch chunks run on
+// their own streams so that they overlap.
+struct HostPipe {
+    std::mutex mu;            // one host call at a time per device
+    bool ready = false;
+    cudaStream_t up = nullptr, run = nullptr, down = nullptr;
+    cudaEvent_t start = nullptr, uploaded[kHostChunks] = {}, computed[kHostChunks] = {};
+};
+
+cudaError_t host_pipe(HostPipe *&hp) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static HostPipe pipes[64];
+    static std::mutex mu;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    hp = &pipes[dev];
+    std::lock_guard<std::mutex> lock(mu);
+    if (hp->ready) return cudaSuccess;
+    const unsigned nb = cudaStreamNonBlocking, nt = cudaEventDisableTiming;
+    if ((e = cudaStreamCreateWithFlags(&hp->up, nb))) return e;
+    if ((e = cudaStreamCreateWithFlags(&hp->run, nb))) return e;
+    if ((e = cudaStreamCreateWithFlags(&hp->down, nb))) return e;
+    if ((e = cudaEventCreateWithFlags(&hp->start, nt))) return e;
+    for (int c = 0; c < kHostChunks; ++c) {
+        if ((e = cudaEventCreateWithFlags(&hp->uploaded[c], nt))) return e;
+        if ((e = cudaEventCreateWithFlags(&hp->computed[c], nt))) return e;
+    }
+    hp->ready = true;
+    return cudaSuccess;
+}
+
+}  // namespace
+
 extern "C" gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambda,
                                             const void *h_wlogit, const void *h_u, void *h_out,
                                             void *d_x, void *d_lambda, void *d_wlogit, void *d_u,
@@ -418,18 +457,40 @@ extern "C" gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambd
     if (!d_x || !d_lambda || !d_wlogit || !d_u || !d_out) return GSPN_ERR_NULL;
     const size_t es = dtype == GSPN_BF16 ? 2 : 4;
     const size_t plane = static_cast<size_t>(H) * W * es;
-    const size_t nx = static_cast<size_t>(B) * Cc * plane;
-    const size_t ng = static_cast<size_t>(B) * 4 * Cc * plane;
-    const size_t nw = static_cast<size_t>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane;
-    if (cudaMemcpyAsync(d_x, h_x, nx, cudaMemcpyHostToDevice, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(d_lambda, h_lambda, ng, cudaMemcpyHostToDevice, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(d_wlogit, h_wlogit, nw, cudaMemcpyHostToDevice, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(d_u, h_u, ng, cudaMemcpyHostToDevice, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    gspn_status st = gspn_prop2d_fwd(d_x, d_lambda, d_wlogit, d_u, B, Cc, H, W, dirs, share_w,
-                                     dtype, d_out, stream);
-    if (st != GSPN_OK) return st;
-    if (cudaMemcpyAsync(h_out, d_out, nx, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    // bytes per batch element of each tensor (the batch is the outer dimension)
+    const size_t bx = static_cast<size_t>(Cc) * plane;
+    const size_t bg = 4 * bx;
+    const size_t bw = static_cast<size_t>(4) * (share_w ? 1 : Cc) * 3 * plane;
+    HostPipe *hp = nullptr;
+    if (host_pipe(hp) != cudaSuccess) return GSPN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(hp->mu);
+    // the pipeline starts after the work already queued on `stream`
+    if (cudaEventRecord(hp->start, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaStreamWaitEvent(hp->up, hp->start, 0) != cudaSuccess) return GSPN_ERR_CUDA;
+    const int nchunk = B < kHostChunks ? B : kHostChunks;
+    auto cb = [](const void *p, size_t off) { return static_cast<const char *>(p) + off; };
+    auto mb = [](void *p, size_t off) { return static_cast<char *>(p) + off; };
+    for (int c = 0; c < nchunk; ++c) {
+        const int b0 = static_cast<int>(static_cast<long long>(B) * c / nchunk);
+        const int b1 = static_cast<int>(static_cast<long long>(B) * (c + 1) / nchunk);
+        const size_t n = static_cast<size_t>(b1 - b0);
+        if (cudaMemcpyAsync(mb(d_x, b0 * bx), cb(h_x, b0 * bx), n * bx, cudaMemcpyHostToDevice, hp->up) ||
+            cudaMemcpyAsync(mb(d_lambda, b0 * bg), cb(h_lambda, b0 * bg), n * bg, cudaMemcpyHostToDevice, hp->up) ||
+            cudaMemcpyAsync(mb(d_wlogit, b0 * bw), cb(h_wlogit, b0 * bw), n * bw, cudaMemcpyHostToDevice, hp->up) ||
+            cudaMemcpyAsync(mb(d_u, b0 * bg), cb(h_u, b0 * bg), n * bg, cudaMemcpyHostToDevice, hp->up) ||
+            cudaEventRecord(hp->uploaded[c], hp->up) || cudaStreamWaitEvent(hp->run, hp->uploaded[c], 0))
+            return GSPN_ERR_CUDA;
+        const gspn_status st = gspn_prop2d_fwd(cb(d_x, b0 * bx), cb(d_lambda, b0 * bg),
+                                               cb(d_wlogit, b0 * bw), cb(d_u, b0 * bg),
+                                               b1 - b0, Cc, H, W, dirs, share_w, dtype,
+                                               mb(d_out, b0 * bx), hp->run);
+        if (st != GSPN_OK) return st;
+        if (cudaEventRecord(hp->computed[c], hp->run) || cudaStreamWaitEvent(hp->down, hp->computed[c], 0) ||
+            cudaMemcpyAsync(mb(h_out, b0 * bx), cb(d_out, b0 * bx), n * bx, cudaMemcpyDeviceToHost, hp->down))
+            return GSPN_ERR_CUDA;
+    }
+    // the downloads wait for every kernel, which waited for every upload
+    if (cudaStreamSynchronize(hp->down) != cudaSuccess) return GSPN_ERR_CUDA;
     return GSPN_OK;
 }
 
