@@ -74,9 +74,25 @@ typedef enum {
     GSPN_ERR_WORKSPACE = 8, /* workspace smaller than gspn_prop2d_workspace_bytes */
     GSPN_ERR_NOALLOC_LIMIT = 9, /* gspn_prop2d_fwd_noalloc: the sizes need more than
                                    GSPN_NOALLOC_WORKSPACE_BYTES of scratch */
-    GSPN_ERR_SHARING = 10  /* gspn_prop2d_fwd_ex: gate_dirs not 1 or 4, or w_groups not a
+    GSPN_ERR_SHARING = 10, /* gspn_prop2d_fwd_ex: gate_dirs not 1 or 4, or w_groups not a
                               divisor of Cc */
+    GSPN_ERR_ALGO = 11     /* gspn_prop2d_fwd_algo: unknown algorithm, or one that cannot
+                              run these sizes */
 } gspn_status;
+
+/* Kernel choice of gspn_prop2d_fwd_algo.  Every algorithm computes the same
+ * Prop2D; they differ in how the work is spread over the GPU. */
+typedef enum {
+    GSPN_ALGO_AUTO = 0,       /* the library's choice, the one every other entry point makes */
+    GSPN_ALGO_DIRECTION = 1,  /* one CTA per plane, one warp per direction (lines <= 256;
+                                 bf16 rows of even width) */
+    GSPN_ALGO_SWEEP_PAIR = 2, /* both sweeps of an orientation in the two halves of a warp
+                                 (lines 2..128; bf16 rows of even width) */
+    GSPN_ALGO_SPLIT = 3,      /* one cluster of four CTAs per plane, one CTA per direction,
+                                 planes staged whole in shared memory (lines 2..128; the six
+                                 planes a direction reads must fit one CTA; bf16 needs H*W even) */
+    GSPN_ALGO_GENERIC = 4     /* the general kernel (lines <= 4096) */
+} gspn_algo;
 
 enum {
     GSPN_DIR_TB = 1,    /* top -> bottom: rows i = 0..H-1, previous row i-1 */
@@ -132,6 +148,19 @@ gspn_status gspn_prop2d_fwd_ex(const void *x, const void *lambda, const void *wl
                                const void *u, int B, int Cc, int H, int W, int dirs,
                                int gate_dirs, int w_groups, gspn_dtype dtype, void *out,
                                cudaStream_t stream);
+
+/*
+ * gspn_prop2d_fwd_algo -- gspn_prop2d_fwd_ex with the kernel named by `algo`
+ * instead of the library's choice (for reproducible benchmarks, and for tests
+ * that must reach one kernel).  GSPN_ALGO_AUTO is gspn_prop2d_fwd_ex.
+ * Returns GSPN_ERR_ALGO, before anything is launched, for an unknown `algo`
+ * or one whose limits (above) the sizes exceed; otherwise arguments and
+ * errors as gspn_prop2d_fwd_ex.
+ */
+gspn_status gspn_prop2d_fwd_algo(const void *x, const void *lambda, const void *wlogit,
+                                 const void *u, int B, int Cc, int H, int W, int dirs,
+                                 int gate_dirs, int w_groups, gspn_dtype dtype, gspn_algo algo,
+                                 void *out, cudaStream_t stream);
 
 /*
  * gspn_prop2d_workspace_bytes -- size of the workspace gspn_prop2d_fwd_ws

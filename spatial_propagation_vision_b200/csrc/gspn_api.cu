@@ -157,6 +157,8 @@ extern "C" const char *gspn_status_str(gspn_status s) {
         case GSPN_ERR_DEVICE: return "GSPN_ERR_DEVICE: the current device is not sm_100";
         case GSPN_ERR_SHARING:
             return "GSPN_ERR_SHARING: gate_dirs must be 1 or 4 and w_groups a divisor of Cc";
+        case GSPN_ERR_ALGO:
+            return "GSPN_ERR_ALGO: unknown algorithm, or one that cannot run these sizes";
         case GSPN_ERR_NOALLOC_LIMIT:
             return "GSPN_ERR_NOALLOC_LIMIT: these sizes need more scratch than the library's "
                    "built-in GSPN_NOALLOC_WORKSPACE_BYTES array";
@@ -203,6 +205,42 @@ DirLaunch dir_variant(int es, const DirPlan &pl, bool pre) {
 // capacity 32 RP + 16 NS.
 constexpr int kMaxPairLine = 128;
 
+// Planes that leave most of the GPU idle when one CTA runs a whole plane go
+// to the cluster-split kernel (one CTA per direction).
+constexpr int kMaxSplitLine = 128;
+
+// Cluster-split kernel (prop2d_split.cuh) when the shape suits it: both sides
+// 2..128, plane byte sizes a multiple of 4 (4-byte tail copies), the six
+// staged planes and the fp32 output plane within one CTA's shared memory.
+// Without `forced`, only when there are fewer planes than SMs (measured on
+// B200; see the routing note in prop2d_run).  `taken` tells whether it was
+// launched.
+cudaError_t try_split(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
+                      int Cc, int H, int W, int dirs, Sharing sh, int es, void *out,
+                      const DeviceProps &dp, cudaStream_t stream, bool forced, bool &taken) {
+    taken = false;
+    const int mx = H > W ? H : W;
+    if (H < 2 || W < 2 || mx > kMaxSplitLine) return cudaSuccess;
+    const long long HW = static_cast<long long>(H) * W;
+    if ((HW * es) % 4 != 0) return cudaSuccess;
+    if (!forced && static_cast<long long>(B) * Cc >= dp.sms) return cudaSuccess;
+    const long long slot = round_up(static_cast<int>(HW * es) + 16, 16);
+    const long long y_off = gspn::kTensors * slot;
+    const long long smem = y_off + round_up(static_cast<int>((HW + 1) * 4), 16);
+    if (smem > dp.smem_optin) return cudaSuccess;
+    if (static_cast<long long>(B) * Cc * gspn::kSplitCluster > 0x7fffffffLL) return cudaSuccess;
+    gspn::SplitParams sp{};
+    sp.x = x; sp.lam = lambda; sp.wl = wlogit; sp.u = u; sp.out = out;
+    sp.B = B; sp.Cc = Cc; sp.H = H; sp.W = W; sp.dirs = dirs;
+    sp.gate_dirs = sh.gate_dirs;
+    sp.w_groups = sh.w_groups;
+    sp.w_cpg = Cc / sh.w_groups;
+    sp.slot = static_cast<int>(slot);
+    sp.y_off = static_cast<int>(y_off);
+    taken = true;
+    return launch_split((mx + 31) / 32, es == 2, sp, static_cast<int>(smem), stream, g_last);
+}
+
 // Sweep-pair kernel (prop2d_pair.cuh) when the shape suits it: both sides
 // 2..128, rows at least as long as the lanes' pair blocks (their words are
 // read straight from global memory), bf16 rows of even width (4-byte aligned
@@ -211,7 +249,7 @@ constexpr int kMaxPairLine = 128;
 // whether it was launched.
 cudaError_t try_pair(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
                      int Cc, int H, int W, int dirs, Sharing sh, int es, void *out,
-                     const DeviceProps &dp, cudaStream_t stream, bool &taken) {
+                     const DeviceProps &dp, cudaStream_t stream, bool forced, bool &taken) {
     taken = false;
     const int mx = H > W ? H : W;
     if (H < 2 || W < 2 || mx > kMaxPairLine || (es == 2 && W % 2)) return cudaSuccess;
@@ -221,7 +259,7 @@ cudaError_t try_pair(const void *x, const void *lambda, const void *wlogit, cons
     // 0.253 ms), slower when column directions take part on longer lines
     // (74 x 74, bf16, four directions: 0.52 vs 0.33 ms; its one column warp
     // per plane runs both column sweeps).  It takes the shapes where it wins.
-    if (mx > 16 && (dirs & 12) != 0) return cudaSuccess;
+    if (!forced && mx > 16 && (dirs & 12) != 0) return cudaSuccess;
     const int bucket = (mx + 15) / 16 - 1;           // 0 .. 7
     const int RP = bucket / 2, NS = bucket % 2 + 1;  // capacity 32 RP + 16 NS >= mx
     if (W < 32 * RP) return cudaSuccess;
@@ -273,7 +311,7 @@ cudaError_t try_pair(const void *x, const void *lambda, const void *wlogit, cons
 // check `dirs` and the sharing arguments.
 gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
                        int Cc, int H, int W, int dirs, Sharing sh, gspn_dtype dtype, void *out,
-                       void *ws, cudaStream_t stream) {
+                       void *ws, cudaStream_t stream, gspn_algo algo = GSPN_ALGO_AUTO) {
     g_last = LaunchInfo{};
     if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
     if (dtype != GSPN_F32 && dtype != GSPN_BF16) return GSPN_ERR_DTYPE;
@@ -295,14 +333,27 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
     const int es = dtype == GSPN_BF16 ? 2 : 4;
     cudaError_t err = cudaSuccess;
     const bool pre = sh.w_groups == 1 && ws;
-    if (!pre) {
+    const bool any = algo == GSPN_ALGO_AUTO;
+    // Routing (GSPN_ALGO_AUTO), from B200 measurements: fewer planes than SMs
+    // run on the cluster-split kernel (16 x 16 x 4 planes, fp32: 0.0xx vs
+    // 0.0124 ms on the sweep-pair kernel); the sweep-pair kernel takes lines
+    // of up to 16 and the row directions alone (see try_pair); the rest runs
+    // on the direction kernel, else the general kernel.
+    if (!pre && (any || algo == GSPN_ALGO_SPLIT)) {
         bool taken = false;
-        err = try_pair(x, lambda, wlogit, u, B, Cc, H, W, dirs, sh, es, out, dp, stream, taken);
+        err = try_split(x, lambda, wlogit, u, B, Cc, H, W, dirs, sh, es, out, dp, stream, !any, taken);
         if (taken) return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+        if (!any) return GSPN_ERR_ALGO;
+    }
+    if (!pre && (any || algo == GSPN_ALGO_SWEEP_PAIR)) {
+        bool taken = false;
+        err = try_pair(x, lambda, wlogit, u, B, Cc, H, W, dirs, sh, es, out, dp, stream, !any, taken);
+        if (taken) return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+        if (!any) return GSPN_ERR_ALGO;
     }
     // bf16 rows of even width keep every row and span 4-byte aligned
     const bool dir_ok = maxline <= kMaxDirLine && H >= 2 && W >= 2 && (es == 4 || (W % 2 == 0));
-    if (dir_ok) {
+    if (dir_ok && (any || algo == GSPN_ALGO_DIRECTION)) {
         const int R = (maxline + 31) / 32;
         DirPlan pl;
         pl.p.x = x; pl.p.lam = lambda; pl.p.wl = wlogit; pl.p.u = u; pl.p.out = out;
@@ -344,6 +395,7 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
             return err == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
         }
     }
+    if (!any && algo != GSPN_ALGO_GENERIC) return GSPN_ERR_ALGO;
     GenericParams gp{};
     gp.x = x; gp.lam = lambda; gp.wl = wlogit; gp.u = u; gp.out = out;
     gp.B = B; gp.Cc = Cc; gp.H = H; gp.W = W; gp.dirs = dirs;
@@ -378,6 +430,19 @@ extern "C" gspn_status gspn_prop2d_fwd_ex(const void *x, const void *lambda, con
         return GSPN_ERR_SHARING;
     return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{gate_dirs, w_groups}, dtype,
                       out, nullptr, stream);
+}
+
+extern "C" gspn_status gspn_prop2d_fwd_algo(const void *x, const void *lambda, const void *wlogit,
+                                            const void *u, int B, int Cc, int H, int W, int dirs,
+                                            int gate_dirs, int w_groups, gspn_dtype dtype,
+                                            gspn_algo algo, void *out, cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (dirs < 1 || dirs > 15) return GSPN_ERR_DIRS;
+    if ((gate_dirs != 1 && gate_dirs != 4) || w_groups < 1 || (Cc > 0 && Cc % w_groups != 0))
+        return GSPN_ERR_SHARING;
+    if (algo < GSPN_ALGO_AUTO || algo > GSPN_ALGO_GENERIC) return GSPN_ERR_ALGO;
+    return prop2d_run(x, lambda, wlogit, u, B, Cc, H, W, dirs, Sharing{gate_dirs, w_groups}, dtype,
+                      out, nullptr, stream, algo);
 }
 
 extern "C" size_t gspn_prop2d_workspace_bytes(int B, int Cc, int H, int W, int dirs, int share_w,

@@ -12,6 +12,7 @@
 #include "prop2d_norm.cuh"
 #include "prop2d_pair.cuh"
 #include "prop2d_bwd.cuh"
+#include "prop2d_split.cuh"
 
 namespace gspn_host {
 
@@ -65,6 +66,11 @@ cudaError_t launch_bwd(const gspn::BwdParams &bp, bool bf16, int smem, const Dev
 
 // Normalised weights of the compact mode into the workspace (one launch).
 cudaError_t launch_norm(const gspn::NormParams &np, bool bf16, const DeviceProps &dp, cudaStream_t s);
+
+// Cluster-split kernel: one cluster of four CTAs (one per direction) per
+// plane; R positions per lane (1..4).
+cudaError_t launch_split(int R, bool bf16, const gspn::SplitParams &sp, int smem, cudaStream_t s,
+                         LaunchInfo &li);
 
 // General kernel; `fits` is false when even one output row does not fit.
 cudaError_t launch_generic(const gspn::GenericParams &gp, bool bf16, const DeviceProps &dp,

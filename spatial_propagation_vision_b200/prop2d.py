@@ -25,7 +25,11 @@ lib = ctypes.CDLL(LIB_PATH)
 GSPN_F32, GSPN_BF16 = 0, 1
 STATUS = {0: "GSPN_OK", 1: "GSPN_ERR_NULL", 2: "GSPN_ERR_SHAPE", 3: "GSPN_ERR_DIRS",
           4: "GSPN_ERR_DTYPE", 5: "GSPN_ERR_ALIGN", 6: "GSPN_ERR_CUDA", 7: "GSPN_ERR_DEVICE",
-          8: "GSPN_ERR_WORKSPACE", 9: "GSPN_ERR_NOALLOC_LIMIT", 10: "GSPN_ERR_SHARING"}
+          8: "GSPN_ERR_WORKSPACE", 9: "GSPN_ERR_NOALLOC_LIMIT", 10: "GSPN_ERR_SHARING",
+          11: "GSPN_ERR_ALGO"}
+
+# kernel choices of gspn_prop2d_fwd_algo (gspn_algo)
+ALGO = {"auto": 0, "direction": 1, "sweep_pair": 2, "split": 3, "generic": 4}
 
 # bytes of the library's built-in scratch array (GSPN_NOALLOC_WORKSPACE_BYTES)
 NOALLOC_WORKSPACE_BYTES = 8 * 1024 * 1024
@@ -38,6 +42,8 @@ lib.gspn_prop2d_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _
 lib.gspn_prop2d_fwd_ws.restype = _i
 lib.gspn_prop2d_fwd_ex.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 8 + [_vp, _vp]
 lib.gspn_prop2d_fwd_ex.restype = _i
+lib.gspn_prop2d_fwd_algo.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 9 + [_vp, _vp]
+lib.gspn_prop2d_fwd_algo.restype = _i
 lib.gspn_prop2d_bwd.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 5
 lib.gspn_prop2d_bwd.restype = _i
 lib.gspn_prop2d_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
@@ -139,11 +145,12 @@ def prop2d_fwd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torc
 def prop2d_fwd_ex(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torch.Tensor,
                   dirs: int = 15, gate_dirs: int = 4, w_groups: int | None = None,
                   out: torch.Tensor | None = None,
-                  stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+                  stream: torch.cuda.Stream | None = None, algo: str | None = None) -> torch.Tensor:
     """Prop2D with wider sharing (gspn_prop2d_fwd_ex): lam, u are
     [B,gate_dirs,Cc,H,W] (gate_dirs 4, or 1 shared by all directions);
     wlogit is [B,4,G,3,H,W] with G = w_groups (default Cc), channel c using
-    logit field c // (Cc // G)."""
+    logit field c // (Cc // G).  `algo` (a key of ALGO) names the kernel
+    (gspn_prop2d_fwd_algo); None is the library's choice."""
     B, Cc, H, W = _dims(x)
     if x.dtype not in _DT:
         raise ValueError(f"unsupported dtype {x.dtype}")
@@ -159,9 +166,15 @@ def prop2d_fwd_ex(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: t
         out = torch.empty((B, Cc, H, W), dtype=x.dtype, device=dev)
     _check("out", out, (B, Cc, H, W), x.dtype, dev)
     with torch.cuda.device(dev):
-        st = lib.gspn_prop2d_fwd_ex(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(), u.data_ptr(),
-                                    B, Cc, H, W, int(dirs), int(gate_dirs), G, _DT[x.dtype],
-                                    out.data_ptr(), _stream_handle(stream))
+        if algo is None:
+            st = lib.gspn_prop2d_fwd_ex(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(), u.data_ptr(),
+                                        B, Cc, H, W, int(dirs), int(gate_dirs), G, _DT[x.dtype],
+                                        out.data_ptr(), _stream_handle(stream))
+        else:
+            st = lib.gspn_prop2d_fwd_algo(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(),
+                                          u.data_ptr(), B, Cc, H, W, int(dirs), int(gate_dirs), G,
+                                          _DT[x.dtype], ALGO[algo], out.data_ptr(),
+                                          _stream_handle(stream))
     if st != 0:
         raise GspnError(st)
     return out

@@ -71,7 +71,7 @@ def test_argument_checks(lib, args, status):
 def test_status_strings(lib):
     lib.gspn_status_str.argtypes = [ctypes.c_int]
     lib.gspn_status_str.restype = ctypes.c_char_p
-    for s in range(11):
+    for s in range(12):
         assert lib.gspn_status_str(s).decode().startswith("GSPN_")
     assert lib.gspn_status_str(99) is not None
 
@@ -133,3 +133,23 @@ def _fwd_ex(lib):
 ])
 def test_ex_argument_checks(lib, args, status):
     assert _fwd_ex(lib)(*args, None) == status
+
+
+def _fwd_algo(lib):
+    f = lib.gspn_prop2d_fwd_algo
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9 + [ctypes.c_void_p] * 2
+    f.restype = ctypes.c_int
+    return f
+
+
+@pytest.mark.parametrize("args,status", [
+    ((P, P, P, P, 1, 4, 8, 8, 15, 4, 4, 0, 5, P), 11),     # unknown algorithm
+    ((P, P, P, P, 1, 4, 8, 8, 15, 4, 4, 0, -1, P), 11),
+    ((P, P, P, P, 1, 4, 8, 8, 15, 2, 4, 0, 3, P), 10),     # sharing checked first
+    ((P, P, P, P, 1, 4, 8, 8, 16, 4, 4, 0, 3, P), 3),      # then the direction mask
+    ((P, P, P, P, -1, 4, 8, 8, 15, 4, 4, 0, 1, P), 2),     # negative B
+    ((None, None, None, None, 0, 4, 8, 8, 15, 4, 4, 0, 2, None), 0),   # empty batch
+])
+def test_algo_argument_checks(lib, args, status):
+    """gspn_prop2d_fwd_algo rejects bad arguments before it touches a device."""
+    assert _fwd_algo(lib)(*args, None) == status

@@ -68,12 +68,36 @@ def workspace(gspn, inp, dirs=15, share_w=1):
     return torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
 
 
-def check(gspn, inp, dirs=15, share_w=0, planes=None, what="", ws=False, path=None):
+# the kernel (gspn_prop2d_fwd_algo) behind each launch path
+ALGO_OF_PATH = {"dir": "direction", "dir-shared": "direction", "dir-yglobal": "direction",
+                "dir-banded": "direction", "pair": "sweep_pair", "split": "split",
+                "generic": "generic"}
+
+
+def check(gspn, inp, dirs=15, share_w=0, planes=None, what="", ws=False, path=None, algo=None,
+          skip_refused=False):
     """Run the library and compare with the oracle; `path`, when given, is the
-    launch path the call must have taken (gspn_last_launch_info)."""
+    launch path the call must have taken (gspn_last_launch_info).  The kernel
+    is pinned to the path's (gspn_prop2d_fwd_algo) unless `algo` says
+    otherwise ("auto": the library's own choice, which `path` then checks);
+    calls with a workspace always make the library's choice.  With
+    `skip_refused`, a kernel that refuses the sizes (GSPN_ERR_ALGO) skips the
+    test."""
     d = to_dev(inp)
-    kw = {"workspace": workspace(gspn, inp, dirs, share_w)} if ws else {}
-    y = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=dirs, share_w=share_w, **kw)
+    if algo is None and path is not None and not ws:
+        algo = ALGO_OF_PATH[path]
+    if ws or algo is None:
+        kw = {"workspace": workspace(gspn, inp, dirs, share_w)} if ws else {}
+        y = gspn.prop2d_fwd(d["x"], d["lam"], d["wlogit"], d["u"], dirs=dirs, share_w=share_w, **kw)
+    else:
+        G = 1 if share_w else inp["x"].shape[1]
+        try:
+            y = gspn.prop2d_fwd_ex(d["x"], d["lam"], d["wlogit"], d["u"], dirs=dirs, w_groups=G,
+                                   algo=algo)
+        except gspn.GspnError as e:
+            if skip_refused and e.status == 11:
+                pytest.skip(f"{algo} does not take {tuple(inp['x'].shape)}")
+            raise
     torch.cuda.synchronize()
     if path is not None:
         assert gspn.launch_info()["path"] == path, (what, gspn.launch_info())
@@ -133,28 +157,35 @@ SHAPES = [
 ]
 
 
+# every kernel on every shape it takes (refusals skip), and the library's choice
+ALGOS = ["auto", "direction", "sweep_pair", "split", "generic"]
+
+
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_shapes(gspn, shape, dtype):
+def test_shapes(gspn, shape, dtype, algo):
     B, Cc, H, W = shape
     inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=hash(shape) % 1000)
-    check(gspn, inp, what=f"{shape} {dtype}")
+    check(gspn, inp, what=f"{shape} {dtype} {algo}", algo=algo, skip_refused=True)
 
 
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("dirs", [1, 2, 4, 8, 3, 12, 5, 10, 6, 9, 7, 11, 13, 14, 15])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_direction_masks(gspn, dirs, dtype):
+def test_direction_masks(gspn, dirs, dtype, algo):
     inp = make_inputs(2, 3, 21, 18, sigma_w=2.0, dtype=dtype, seed=dirs)
-    check(gspn, inp, dirs=dirs, what=f"dirs={dirs}")
+    check(gspn, inp, dirs=dirs, what=f"dirs={dirs} {algo}", algo=algo, skip_refused=True)
 
 
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", [(2, 5, 16, 16), (3, 4, 37, 38), (1, 3, 148, 148)],
                          ids=lambda s: "x".join(map(str, s)))
-def test_share_w(gspn, shape, dtype):
+def test_share_w(gspn, shape, dtype, algo):
     B, Cc, H, W = shape
     inp = make_inputs(B, Cc, H, W, share_w=1, sigma_w=1.0, dtype=dtype, seed=7)
-    check(gspn, inp, share_w=1, what=f"share_w {shape}")
+    check(gspn, inp, share_w=1, what=f"share_w {shape} {algo}", algo=algo, skip_refused=True)
 
 
 # --------------------------------------------------------------------------
@@ -226,17 +257,27 @@ def test_workspace_unused_without_share_w(gspn):
 # numerics edge cases
 # --------------------------------------------------------------------------
 
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_hand_examples(gspn, dtype):
+def test_hand_examples(gspn, dtype, algo):
+    ran = 0
     for ex in pins.parse_hand_examples():
         x, lam, wl, u = pins.hand_example_inputs(ex)
         inp = {"x": torch.tensor(x, dtype=dtype), "lam": torch.tensor(lam, dtype=dtype),
                "wlogit": torch.tensor(wl, dtype=dtype), "u": torch.tensor(u, dtype=dtype)}
-        check(gspn, inp, dirs=ex["dirs"][0], what=ex["name"])
+        try:
+            check(gspn, inp, dirs=ex["dirs"][0], what=f"{ex['name']} {algo}", algo=algo,
+                  skip_refused=True)
+            ran += 1
+        except pytest.skip.Exception:
+            pass
+    if not ran:
+        pytest.skip(f"{algo} takes none of the hand examples")
 
 
 @pytest.mark.parametrize("dtype,shape,path", [
     ("f32", (1, 2, 19, 23), "dir"), ("bf16", (1, 2, 19, 24), "dir-shared"),
+    ("f32", (1, 2, 19, 23), "split"), ("bf16", (1, 2, 19, 24), "split"),
     ("bf16", (1, 2, 74, 74), "dir-shared"), ("f32", (1, 2, 16, 16), "pair"),
     ("bf16", (1, 2, 16, 16), "pair"), ("f32", (1, 2, 19, 150), "dir"),
     ("bf16", (1, 2, 19, 150), "dir-shared"), ("bf16", (1, 2, 19, 23), "generic")],
@@ -274,6 +315,8 @@ def test_extreme_logits(gspn, mode, dtype, shape, path):
 
 @pytest.mark.parametrize("dtype,shape,path", [
     ("f32", (1, 2, 16, 15), "pair"), ("bf16", (2, 3, 74, 74), "dir-shared"),
+    ("f32", (1, 2, 16, 15), "split"), ("bf16", (2, 3, 74, 74), "split"),
+    ("f32", (1, 2, 60, 100), "split"),
     ("f32", (1, 2, 37, 38), "dir"), ("f32", (1, 2, 19, 150), "dir"),
     ("bf16", (1, 2, 148, 148), "dir-shared"), ("f32", (1, 1, 256, 256), "dir-yglobal"),
     ("bf16", (1, 2, 19, 23), "generic")],
@@ -299,26 +342,53 @@ def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "dir-shared"),
-    ((2, 3, 74, 74), "f32", "dir"),
-    ((4, 4, 37, 37), "f32", "dir"),
-    ((1, 4, 16, 16), "f32", "pair"),
-    ((2, 2, 16, 14), "bf16", "pair"),
-    ((1, 2, 100, 16), "f32", "dir"),           # rows shorter than the pair blocks
-    ((1, 2, 160, 160), "f32", "dir-shared"),   # two output planes do not fit
+    ((2, 3, 74, 74), "bf16", "split"),         # fewer planes than SMs
+    ((2, 3, 74, 74), "f32", "split"),
+    ((4, 4, 37, 37), "f32", "split"),
+    ((1, 4, 16, 16), "f32", "split"),
+    ((2, 2, 16, 14), "bf16", "split"),
+    ((1, 2, 20, 33), "bf16", "split"),         # odd bf16 row width
+    ((8, 24, 16, 16), "f32", "pair"),          # lines of up to 16
+    ((8, 24, 16, 14), "bf16", "pair"),
+    ((4, 40, 37, 37), "f32", "dir"),
+    ((4, 40, 74, 74), "bf16", "dir-shared"),
+    ((4, 40, 20, 33), "bf16", "generic"),      # odd bf16 row width
+    ((1, 2, 160, 160), "f32", "dir-shared"),   # lines over 128; two output planes do not fit
     ((1, 2, 256, 256), "f32", "dir-yglobal"),
     ((1, 2, 256, 256), "bf16", "dir-banded"),
     ((1, 2, 148, 148), "bf16", "dir-shared"),
-    ((1, 2, 20, 33), "bf16", "generic"),       # odd bf16 row width
     ((1, 1, 300, 40), "f32", "generic"),       # line longer than 256
     ((2, 2, 1, 40), "bf16", "generic"),        # lines of one position
     ((1, 3, 17, 1), "f32", "generic"),
-])
+], ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 def test_launch_paths(gspn, shape, dtype, path):
+    """The library's own choice of kernel (and its parity there)."""
     B, Cc, H, W = shape
     inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=11)
-    check(gspn, inp, what=path)
-    assert gspn.launch_info()["path"] == path
+    check(gspn, inp, what=path, path=path, algo="auto")
+
+
+@pytest.mark.parametrize("shape,dtype,algo", [
+    ((1, 2, 200, 40), "f32", "split"),        # line over 128
+    ((1, 2, 15, 15), "bf16", "split"),        # plane of an odd number of bf16 elements
+    ((1, 2, 200, 40), "f32", "sweep_pair"),   # line over 128
+    ((1, 2, 16, 15), "bf16", "sweep_pair"),   # odd bf16 row width
+    ((1, 2, 100, 16), "f32", "sweep_pair"),   # rows shorter than the lanes' pair blocks
+    ((1, 2, 20, 33), "bf16", "direction"),    # odd bf16 row width
+    ((1, 2, 1, 40), "f32", "direction"),      # lines of one position
+    ((1, 2, 300, 40), "bf16", "direction")],  # line over 256
+    ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_algo_refused_when_out_of_range(gspn, shape, dtype, algo):
+    """A named kernel whose limits the sizes exceed is refused (GSPN_ERR_ALGO)
+    before anything runs: the output is left untouched."""
+    B, Cc, H, W = shape
+    inp = to_dev(make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=5))
+    out = torch.full_like(inp["x"], 7.0)
+    with pytest.raises(gspn.GspnError) as e:
+        gspn.prop2d_fwd_ex(inp["x"], inp["lam"], inp["wlogit"], inp["u"], algo=algo, out=out)
+    torch.cuda.synchronize()
+    assert e.value.status == 11
+    assert bool((out == 7.0).all())
 
 
 def test_host_entry_point(gspn):
@@ -370,6 +440,7 @@ def test_output_fully_overwritten(gspn):
 
 @pytest.mark.parametrize("dtype,shape,path", [
     ("bf16", (2, 4, 74, 74), "dir-shared"), ("f32", (1, 6, 16, 16), "pair"),
+    ("bf16", (2, 4, 74, 74), "split"), ("f32", (1, 4, 37, 38), "split"),
     ("f32", (1, 4, 19, 150), "dir"), ("bf16", (1, 4, 19, 150), "dir-shared"),
     ("bf16", (1, 4, 20, 33), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
@@ -385,7 +456,8 @@ def test_sharing_variants(gspn, dtype, shape, path, gate_dirs, groups):
     u = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
     inp = {k: v.to(td) for k, v in {"x": x, "lam": lam, "wlogit": wl, "u": u}.items()}
     d = to_dev(inp)
-    y = gspn.prop2d_fwd_ex(d["x"], d["lam"], d["wlogit"], d["u"], gate_dirs=gate_dirs, w_groups=G)
+    y = gspn.prop2d_fwd_ex(d["x"], d["lam"], d["wlogit"], d["u"], gate_dirs=gate_dirs, w_groups=G,
+                           algo=ALGO_OF_PATH[path])
     torch.cuda.synchronize()
     assert gspn.launch_info()["path"] == path
     yo = oracle.prop2d_ex(f64(inp["x"]), f64(inp["lam"]), f64(inp["wlogit"]), f64(inp["u"]),
