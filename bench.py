@@ -65,7 +65,8 @@ def kernel_sources_sha() -> str:
 
 KERNEL_OF_PATH = {"pair": "prop2d_pair_kernel", "dir": "prop2d_dir_kernel",
                   "dir-shared": "prop2d_dir_kernel", "dir-yglobal": "prop2d_dir_kernel",
-                  "dir-banded": "prop2d_dir_kernel", "generic": "prop2d_generic_kernel"}
+                  "dir-banded": "prop2d_dir_kernel", "dir-half": "prop2d_dir_kernel",
+                  "split": "prop2d_split_kernel", "generic": "prop2d_generic_kernel"}
 
 
 def profile_path(kernel: str, workload: str) -> str:

@@ -18,6 +18,13 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
     return __float2bfloat16_rn(v);
 }
 
+// Two fp32 values rounded to bf16 (round to nearest even) in one 32-bit word:
+// x in the low half, y in the high half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t *>(&b);
+}
+
 // ---------------------------------------------------------------------------
 // hardware approximations: 2^x and 1/x (flush-to-zero), byte permutation
 // ---------------------------------------------------------------------------

@@ -23,6 +23,7 @@ cudaError_t launch_dir_t(const DirPlan &pl, const DeviceProps &dp, cudaStream_t 
     li.path = MODE == gspn::kYGlobal   ? "dir-yglobal"
               : MODE == gspn::kYBanded ? "dir-banded"
               : MODE == gspn::kYShared ? "dir-shared"
+              : MODE == gspn::kYHalf   ? "dir-half"
                                        : "dir";
     return cudaGetLastError();
 }

@@ -111,7 +111,15 @@ bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
     // a plane holds its rows plus one dummy row (written by the column lanes
     // past the end of a column or outside the band)
     int band_rows = H, plane_bytes = 0;
-    if (mode == 0 || mode == 3) {
+    // mode 4 (bf16 planes of pair words): W / 2 words and a dummy per row
+    const int YPW = W / 2 + 1;
+    if (mode == 4) {
+        // the two column sweeps meet at a word boundary: each needs at least
+        // one word on its side (W >= 4), or one of them would never reach
+        // the midpoint barrier
+        if (W < 4 || W % 2) return false;
+        plane_bytes = round_up((H + 1) * YPW * 4, 16);
+    } else if (mode == 0 || mode == 3) {
         plane_bytes = round_up((H + 1) * YP * 4, 16);
     } else if (mode == 2) {
         if (cap - rings < n_planes * 2 * YP * 4) return false;
@@ -131,12 +139,13 @@ bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
         off += col_ring;
     }
     p.bar_off = off;
-    p.y_pitch = YP;
+    p.y_pitch = mode == 4 ? YPW : YP;
     p.band_rows = band_rows;
     p.bands = (H + band_rows - 1) / band_rows;
     pl.smem = y_bytes + rings;
     pl.y_global = mode == 1;
     pl.y_shared = mode == 3;
+    pl.y_half = mode == 4;
     return true;
 }
 
@@ -196,6 +205,7 @@ DirLaunch dir_variant(int es, const DirPlan &pl, bool pre) {
         if (pl.y_shared) return pre ? launch_dir_f32_shared_pre : launch_dir_f32_shared;
         return pre ? launch_dir_f32_smem_pre : launch_dir_f32_smem;
     }
+    if (pl.y_half) return pre ? launch_dir_bf16_half_pre : launch_dir_bf16_half;
     if (pl.y_shared) return pre ? launch_dir_bf16_shared_pre : launch_dir_bf16_shared;
     return pre ? launch_dir_bf16_banded_pre : launch_dir_bf16_banded;
 }
@@ -212,9 +222,14 @@ constexpr int kMaxSplitLine = 128;
 // Cluster-split kernel (prop2d_split.cuh) when the shape suits it: both sides
 // 2..128, plane byte sizes a multiple of 4 (4-byte tail copies), the six
 // staged planes and the fp32 output plane within one CTA's shared memory.
-// Without `forced`, only when there are fewer planes than SMs (measured on
-// B200; see the routing note in prop2d_run).  `taken` tells whether it was
-// launched.
+// Without `forced`, only for fewer planes than twice the SM count (than the
+// SM count for lines of up to 16, where the sweep-pair kernel is quick) whose
+// CTAs (four per plane) run in at most two waves.  Measured on B200 (device time
+// per call, CUDA graphs, split vs the best other kernel): 16 x 16 x 4 planes
+// fp32 4.9 vs 6.9 us; 74 x 74 bf16, 64 planes 22 vs 50 us, 128 planes 42 vs
+// 50 us, 256 planes (four waves) 83 vs 54 us; 37 x 37 fp32, 256 planes 21 vs
+// 24 us, 512 planes (three waves) 32 vs 29 us; 16 x 16 fp32, 512 planes 15 vs
+// 8 us.  `taken` tells whether it was launched.
 cudaError_t try_split(const void *x, const void *lambda, const void *wlogit, const void *u, int B,
                       int Cc, int H, int W, int dirs, Sharing sh, int es, void *out,
                       const DeviceProps &dp, cudaStream_t stream, bool forced, bool &taken) {
@@ -223,11 +238,18 @@ cudaError_t try_split(const void *x, const void *lambda, const void *wlogit, con
     if (H < 2 || W < 2 || mx > kMaxSplitLine) return cudaSuccess;
     const long long HW = static_cast<long long>(H) * W;
     if ((HW * es) % 4 != 0) return cudaSuccess;
-    if (!forced && static_cast<long long>(B) * Cc >= dp.sms) return cudaSuccess;
+    const long long planes = static_cast<long long>(B) * Cc;
+    if (!forced && (planes >= 2LL * dp.sms || (planes >= dp.sms && mx <= 16))) return cudaSuccess;
     const long long slot = round_up(static_cast<int>(HW * es) + 16, 16);
     const long long y_off = gspn::kTensors * slot;
     const long long smem = y_off + round_up(static_cast<int>((HW + 1) * 4), 16);
     if (smem > dp.smem_optin) return cudaSuccess;
+    const int R = (mx + 31) / 32;
+    if (!forced) {
+        int per_sm = 0;
+        if (split_occupancy(R, es == 2, static_cast<int>(smem), per_sm) != cudaSuccess) return cudaSuccess;
+        if (planes * gspn::kSplitCluster > 2LL * dp.sms * per_sm) return cudaSuccess;
+    }
     if (static_cast<long long>(B) * Cc * gspn::kSplitCluster > 0x7fffffffLL) return cudaSuccess;
     gspn::SplitParams sp{};
     sp.x = x; sp.lam = lambda; sp.wl = wlogit; sp.u = u; sp.out = out;
@@ -238,7 +260,7 @@ cudaError_t try_split(const void *x, const void *lambda, const void *wlogit, con
     sp.slot = static_cast<int>(slot);
     sp.y_off = static_cast<int>(y_off);
     taken = true;
-    return launch_split((mx + 31) / 32, es == 2, sp, static_cast<int>(smem), stream, g_last);
+    return launch_split(R, es == 2, sp, static_cast<int>(smem), stream, g_last);
 }
 
 // Sweep-pair kernel (prop2d_pair.cuh) when the shape suits it: both sides
@@ -334,9 +356,8 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
     cudaError_t err = cudaSuccess;
     const bool pre = sh.w_groups == 1 && ws;
     const bool any = algo == GSPN_ALGO_AUTO;
-    // Routing (GSPN_ALGO_AUTO), from B200 measurements: fewer planes than SMs
-    // run on the cluster-split kernel (16 x 16 x 4 planes, fp32: 0.0xx vs
-    // 0.0124 ms on the sweep-pair kernel); the sweep-pair kernel takes lines
+    // Routing (GSPN_ALGO_AUTO), from B200 measurements: few planes run on the
+    // cluster-split kernel (see try_split); the sweep-pair kernel takes lines
     // of up to 16 and the row directions alone (see try_pair); the rest runs
     // on the direction kernel, else the general kernel.
     if (!pre && (any || algo == GSPN_ALGO_SPLIT)) {
@@ -369,8 +390,8 @@ gspn_status prop2d_run(const void *x, const void *lambda, const void *wlogit, co
         // bf16: one plane with shared atomics (the four directions run
         // uncoupled until the end of an item), else bands; fp32: two planes
         // (atomic-free), one plane, else global atomics (which always fit)
-        const int order_bf16[2] = {3, 2}, order_f32[3] = {0, 3, 1};
-        const int n_order = es == 2 ? 2 : 3;
+        const int order_bf16[3] = {4, 3, 2}, order_f32[3] = {0, 3, 1};
+        const int n_order = 3;
         for (int oi = 0; oi < n_order && !fit; ++oi) {
             const int mode = es == 2 ? order_bf16[oi] : order_f32[oi];
             for (int ci = 0; ci < 4 && !fit; ++ci) {

@@ -30,6 +30,7 @@ struct DeviceProps {
 struct DirPlan {
     bool y_global = false;
     bool y_shared = false;   // one plane, shared-memory atomics
+    bool y_half = false;     // two bf16 planes of pair words, no atomics
     int smem = 0;
     gspn::DirParams p{};
 };
@@ -48,6 +49,8 @@ cudaError_t launch_dir_bf16_banded(int R, const DirPlan &pl, const DeviceProps &
 cudaError_t launch_dir_bf16_banded_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_shared(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 cudaError_t launch_dir_bf16_shared_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_half(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
+cudaError_t launch_dir_bf16_half_pre(int R, const DirPlan &pl, const DeviceProps &dp, cudaStream_t s, LaunchInfo &li);
 
 // Sweep-pair kernel: RP position pairs and NS single positions per lane.
 cudaError_t launch_pair_bf16(int RP, int NS, const gspn::PairParams &pp, int smem,
@@ -71,6 +74,8 @@ cudaError_t launch_norm(const gspn::NormParams &np, bool bf16, const DeviceProps
 // plane; R positions per lane (1..4).
 cudaError_t launch_split(int R, bool bf16, const gspn::SplitParams &sp, int smem, cudaStream_t s,
                          LaunchInfo &li);
+// Resident CTAs per SM of that kernel with `smem` bytes (cached).
+cudaError_t split_occupancy(int R, bool bf16, int smem, int &per_sm);
 
 // General kernel; `fits` is false when even one output row does not fit.
 cudaError_t launch_generic(const gspn::GenericParams &gp, bool bf16, const DeviceProps &dp,

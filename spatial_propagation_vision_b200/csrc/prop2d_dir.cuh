@@ -74,6 +74,9 @@ constexpr int kYGlobal = 2;   // fp32 output accumulated in global memory (L2 at
 constexpr int kYShared = 3;   // one fp32 plane in shared memory for all four directions
                               // (shared-memory atomics; the warps never wait for one
                               // another before the end of a plane)
+constexpr int kYHalf = 4;     // bf16 only: two bf16 planes (rows, columns) of pair words
+                              // (columns 2j, 2j+1 in word j), written without atomics:
+                              // each sweep pair splits at a word-aligned midpoint
 
 struct DirParams {
     const void *x, *lam, *wl, *u;
@@ -86,7 +89,8 @@ struct DirParams {
     int ring[4];                // byte offset of column direction d's ring (-1: none)
     int bar_off;                // byte offset of the column warps' plane-pointer tables
     int ycol_off;               // byte offset of the column directions' output plane
-    int y_pitch;                // floats per staged output row (odd, > every ycol(j), j < W)
+    int y_pitch;                // floats per staged output row (odd, > every ycol(j), j < W);
+                                // kYHalf: 32-bit words per row (>= W/2 + 1, the last a dummy)
     unsigned long long end_x, end_gate, end_wl;   // byte sizes of x, lambda/u, logits
 };
 
@@ -355,6 +359,8 @@ struct RowScan {
     long long pf_cur, pf_next;
     const bool fwd;             // top-down (else bottom-up)
     const int split;            // first step after the midpoint (see sweep_split)
+    int hw[NP > 0 ? NP : 1];    // kYHalf: word of each position pair in a plane row
+    int hs;                     // kYHalf: byte of the single position in a plane row
 
     __device__ static int pos(int lane, int r) {
         return r < 2 * NP ? 64 * (r / 2) + 2 * lane + (r & 1) : 64 * NP + lane;
@@ -373,6 +379,13 @@ struct RowScan {
             g.thr[r] = __float_as_int((q > 0 && q + 1 < W) ? 1e11f : 1e5f);
             // positions past the row end write the plane's last (dummy) column
             cs[r] = q < W ? q ^ ((q >> 5) & 1) : p_.y_pitch - 1;
+        }
+        if (MODE == kYHalf) {
+            // pairs past the row end write the dummy word; a single past the
+            // end writes the dummy word's half of the lane's parity
+#pragma unroll
+            for (int k = 0; k < (NP > 0 ? NP : 1); ++k) hw[k] = 64 * k + 2 * lane_ < W ? 32 * k + lane_ : p_.y_pitch - 1;
+            hs = 64 * NP + lane_ < W ? 4 * (32 * NP) + 2 * lane_ : 4 * (p_.y_pitch - 1) + 2 * (lane_ & 1);
         }
 #pragma unroll
         for (int k = 0; k < kWords; ++k) {
@@ -460,15 +473,35 @@ struct RowScan {
                                          float *yg, int band_lo, int band_hi, bool first) const {
         const bool in = MODE != kYBanded || (row >= band_lo && row < band_hi);
         float *yl = ys + (row - band_lo) * p.y_pitch;
+        if constexpr (MODE == kYHalf) {
+            uint32_t *wl = reinterpret_cast<uint32_t *>(yl);
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const float cy = W.uu[r] * h[r];
-            if (MODE == kYGlobal) {
-                if (g.valid[r]) atomicAdd(yg + static_cast<size_t>(row) * p.W + pos(lane, r), cy);
-            } else if (MODE == kYShared) {
-                if (g.valid[r] && in) atomicAdd(yl + cs[r], cy);
-            } else {
-                if (in) put_y(yl + cs[r], cy, first);
+            for (int k = 0; k < NP; ++k) {
+                float2 v = make_float2(W.uu[2 * k] * h[2 * k], W.uu[2 * k + 1] * h[2 * k + 1]);
+                if (!first) {
+                    const uint32_t o = wl[hw[k]];
+                    v.x += __uint_as_float(o << 16);
+                    v.y += __uint_as_float(o & 0xffff0000u);
+                }
+                wl[hw[k]] = pack_bf16x2(v);
+            }
+            if (kSingle) {
+                unsigned short *a = reinterpret_cast<unsigned short *>(reinterpret_cast<unsigned char *>(yl) + hs);
+                float v = W.uu[R - 1] * h[R - 1];
+                if (!first) v += __uint_as_float(static_cast<uint32_t>(*a) << 16);
+                *a = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float cy = W.uu[r] * h[r];
+                if (MODE == kYGlobal) {
+                    if (g.valid[r]) atomicAdd(yg + static_cast<size_t>(row) * p.W + pos(lane, r), cy);
+                } else if (MODE == kYShared) {
+                    if (g.valid[r] && in) atomicAdd(yl + cs[r], cy);
+                } else {
+                    if (in) put_y(yl + cs[r], cy, first);
+                }
             }
         }
     }
@@ -592,7 +625,8 @@ struct ColScan {
     LaneGeom<R> g;
     int rowq[R];        // byte offset of strip row q_r in a stage (row 0 when q_r >= H)
     bool inb[R];        // q_r is an output row of the current item
-    int yoff[R];        // offset (floats) of its output row in the column plane
+    int yoff[R];        // offset (floats; kYHalf: words) of its output row in the column plane
+    float held[R];      // kYHalf: outputs of the first column of a word pair
     int issue_item;
     const char **gtab;  // [kTensors] planes of the item being issued (shared memory)
     const bool fwd;     // left-right (else right-left)
@@ -606,7 +640,10 @@ struct ColScan {
                        (kColStrip / static_cast<int>(sizeof(T)))),
           total_chunks(0), issue_item(-1),
           gtab(reinterpret_cast<const char **>(smem + p_.bar_off + 128 + 64 * (d - 2))),
-          fwd(d == 2), split(sweep_split((p_.dirs & 12) == 12, d == 2, p_.W)),
+          fwd(d == 2),
+          split(MODE == kYHalf && (p_.dirs & 12) == 12
+                    ? (d == 2 ? 2 * ((p_.W / 2 + 1) / 2) : 2 * ((p_.W / 2) / 2))
+                    : sweep_split((p_.dirs & 12) == 12, d == 2, p_.W)),
           // bf16 word -> float of its first / second column in scan order:
           // the low half (bits << 16) or the high half (bits & 0xffff0000)
           selA(d == 2 ? 0x1044u : 0x3244u), selB(d == 2 ? 0x3244u : 0x1044u) {
@@ -738,6 +775,30 @@ struct ColScan {
             }
     }
 
+    // kYHalf: the first column of a word pair (scan order) is held, the
+    // second stores the pair (LR: columns 2j, 2j+1; RL: 2j+1, 2j).
+    template <int J>
+    __device__ __forceinline__ void emit_half(const float (&h)[R], const LineW<R> &W, int col, float *ys,
+                                              bool first) {
+        if constexpr ((J & 1) == 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) held[r] = W.uu[r] * h[r];
+        } else {
+            uint32_t *yw = reinterpret_cast<uint32_t *>(ys) + (col >> 1);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float cur = W.uu[r] * h[r];
+                float2 v = fwd ? make_float2(held[r], cur) : make_float2(cur, held[r]);
+                if (!first) {
+                    const uint32_t o = yw[yoff[r]];
+                    v.x += __uint_as_float(o << 16);
+                    v.y += __uint_as_float(o & 0xffff0000u);
+                }
+                yw[yoff[r]] = pack_bf16x2(v);
+            }
+        }
+    }
+
     __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int col, float *ys,
                                          float *yg, bool first) const {
         const int yc = ycol(col);
@@ -800,7 +861,8 @@ struct ColScan {
             }
         }
         const bool bad = next_weights<PRE>(v, g, Wb[(J + 1) & 1]);
-        emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
+        if constexpr (MODE == kYHalf) emit_half<J>(h, Wc, fwd ? st : L - 1 - st, ys, st < split);
+        else emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
         if (!PRE) line_terms_fix(bad, v, g, Wb[(J + 1) & 1]);
         if (MODE != kYGlobal && MODE != kYShared && st + 1 == split) pair_barrier(3);
     }
@@ -891,19 +953,43 @@ __device__ __forceinline__ void dir_role(const DirParams &p, unsigned char *smem
             // position of a plane is stored again by the next item
             T *outp = static_cast<T *>(p.out) + static_cast<size_t>(plane) * p.H * p.W +
                       static_cast<size_t>(band_lo) * p.W;
-            for (int i = warp; i < band_hi - band_lo; i += 4) {
-                float *yr = ysr + i * YP;
-                const float *yc = ysc + i * YP;
-                T *orow = outp + static_cast<size_t>(i) * p.W;
-                for (int j = lane; j < p.W; j += 32) {
-                    const int c = ycol(j);
-                    if (MODE == kYShared) {
-                        // the single plane is accumulated into: clear it
-                        orow[j] = from_f<T>(yr[c]);
-                        yr[c] = 0.0f;
-                    } else {
-                        const float v = (has_row ? yr[c] : 0.0f) + (has_col ? yc[c] : 0.0f);
-                        orow[j] = from_f<T>(v);
+            if constexpr (MODE == kYHalf) {
+                // word j of a plane row holds columns 2j, 2j+1 (W is even)
+                const uint32_t *wr = reinterpret_cast<const uint32_t *>(ysr);
+                const uint32_t *wc = reinterpret_cast<const uint32_t *>(ysc);
+                uint32_t *ow = reinterpret_cast<uint32_t *>(outp);
+                const int nw = p.W / 2;
+                for (int i = warp; i < p.H; i += 4) {
+                    for (int j = lane; j < nw; j += 32) {
+                        float2 v = make_float2(0.0f, 0.0f);
+                        if (has_row) {
+                            const uint32_t o = wr[i * YP + j];
+                            v.x += __uint_as_float(o << 16);
+                            v.y += __uint_as_float(o & 0xffff0000u);
+                        }
+                        if (has_col) {
+                            const uint32_t o = wc[i * YP + j];
+                            v.x += __uint_as_float(o << 16);
+                            v.y += __uint_as_float(o & 0xffff0000u);
+                        }
+                        ow[static_cast<size_t>(i) * nw + j] = pack_bf16x2(v);
+                    }
+                }
+            } else {
+                for (int i = warp; i < band_hi - band_lo; i += 4) {
+                    float *yr = ysr + i * YP;
+                    const float *yc = ysc + i * YP;
+                    T *orow = outp + static_cast<size_t>(i) * p.W;
+                    for (int j = lane; j < p.W; j += 32) {
+                        const int c = ycol(j);
+                        if (MODE == kYShared) {
+                            // the single plane is accumulated into: clear it
+                            orow[j] = from_f<T>(yr[c]);
+                            yr[c] = 0.0f;
+                        } else {
+                            const float v = (has_row ? yr[c] : 0.0f) + (has_col ? yc[c] : 0.0f);
+                            orow[j] = from_f<T>(v);
+                        }
                     }
                 }
             }

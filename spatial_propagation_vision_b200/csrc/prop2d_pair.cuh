@@ -298,10 +298,6 @@ __device__ __forceinline__ void pair_recur(PairState<RP, NS> &S, const PairTerms
 // the input/output element type: fp32, or bf16 for bf16 inputs (the sum of
 // two directions rounded to bf16 once per sweep; the final sum of the two
 // planes is formed in fp32).
-__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(v.x, v.y);
-    return *reinterpret_cast<const uint32_t *>(&b);
-}
 
 template <int RP, int NS, bool ADD>
 __device__ __forceinline__ void pair_emit(float *Y, int hl, const PairState<RP, NS> &S,

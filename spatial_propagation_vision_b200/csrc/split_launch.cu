@@ -35,7 +35,24 @@ cudaError_t launch_split_r(int R, const gspn::SplitParams &sp, int smem, cudaStr
     }
 }
 
+template <typename T>
+const void *split_kernel_ptr(int R) {
+    switch (R) {
+        case 1: return reinterpret_cast<const void *>(gspn::prop2d_split_kernel<T, 1>);
+        case 2: return reinterpret_cast<const void *>(gspn::prop2d_split_kernel<T, 2>);
+        case 3: return reinterpret_cast<const void *>(gspn::prop2d_split_kernel<T, 3>);
+        case 4: return reinterpret_cast<const void *>(gspn::prop2d_split_kernel<T, 4>);
+        default: return nullptr;
+    }
+}
+
 }  // namespace
+
+cudaError_t split_occupancy(int R, bool bf16, int smem, int &per_sm) {
+    const void *k = bf16 ? split_kernel_ptr<__nv_bfloat16>(R) : split_kernel_ptr<float>(R);
+    if (!k) return cudaErrorInvalidValue;
+    return kernel_occupancy(k, gspn::kSplitThreads, smem, per_sm);
+}
 
 cudaError_t launch_split(int R, bool bf16, const gspn::SplitParams &sp, int smem, cudaStream_t s,
                          LaunchInfo &li) {

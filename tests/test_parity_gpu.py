@@ -70,6 +70,7 @@ def workspace(gspn, inp, dirs=15, share_w=1):
 
 # the kernel (gspn_prop2d_fwd_algo) behind each launch path
 ALGO_OF_PATH = {"dir": "direction", "dir-shared": "direction", "dir-yglobal": "direction",
+                "dir-half": "direction",
                 "dir-banded": "direction", "pair": "sweep_pair", "split": "split",
                 "generic": "generic"}
 
@@ -129,7 +130,7 @@ def test_workload_full(gspn, name):
     print(f"\n{name}: max|err| / max|y| = {rel:.3e}")
 
 
-@pytest.mark.parametrize("name,path", [("1k", "dir-shared"), ("2k", "dir-shared"),
+@pytest.mark.parametrize("name,path", [("1k", "dir-half"), ("2k", "dir-half"),
                                        ("orig", "dir-yglobal")])
 def test_workload_all_planes(gspn, name, path):
     """Full-size workload in the launch the benchmark times, every plane
@@ -196,7 +197,7 @@ def test_workload_2k_workspace(gspn):
     """The 2k compact workload through gspn_prop2d_fwd_ws (every plane)."""
     w = WORKLOADS["2k"]
     inp = workload_inputs(w, seed=0)
-    rel = check(gspn, inp, share_w=1, planes="all", what="2k ws", ws=True, path="dir-shared")
+    rel = check(gspn, inp, share_w=1, planes="all", what="2k ws", ws=True, path="dir-half")
     print(f"\n2k with workspace (all planes): max|err| / max|y| = {rel:.3e}")
     assert gspn.launch_info()["launches"] == 2
 
@@ -238,7 +239,7 @@ def test_share_w_workspace_extremes(gspn, mode, dtype, W):
     td = torch.bfloat16 if dtype == "bf16" else torch.float32
     inp = {k: v.to(td) for k, v in inp.items()}
     check(gspn, inp, share_w=1, what=f"ws {mode} {dtype}", ws=True,
-          path="dir-shared" if dtype == "bf16" else "dir")
+          path="dir-half" if dtype == "bf16" else "dir")
     assert gspn.launch_info()["launches"] == 2
 
 
@@ -276,11 +277,12 @@ def test_hand_examples(gspn, dtype, algo):
 
 
 @pytest.mark.parametrize("dtype,shape,path", [
-    ("f32", (1, 2, 19, 23), "dir"), ("bf16", (1, 2, 19, 24), "dir-shared"),
+    ("f32", (1, 2, 19, 23), "dir"), ("bf16", (1, 2, 19, 24), "dir-half"),
+    ("bf16", (1, 2, 19, 2), "dir-shared"),
     ("f32", (1, 2, 19, 23), "split"), ("bf16", (1, 2, 19, 24), "split"),
-    ("bf16", (1, 2, 74, 74), "dir-shared"), ("f32", (1, 2, 16, 16), "pair"),
+    ("bf16", (1, 2, 74, 74), "dir-half"), ("f32", (1, 2, 16, 16), "pair"),
     ("bf16", (1, 2, 16, 16), "pair"), ("f32", (1, 2, 19, 150), "dir"),
-    ("bf16", (1, 2, 19, 150), "dir-shared"), ("bf16", (1, 2, 19, 23), "generic")],
+    ("bf16", (1, 2, 19, 150), "dir-half"), ("bf16", (1, 2, 19, 23), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 @pytest.mark.parametrize("mode", ["all_very_negative", "clamp_binds", "overflow_pairs",
                                   "saturated_positive", "mixed_extremes"])
@@ -314,11 +316,12 @@ def test_extreme_logits(gspn, mode, dtype, shape, path):
 
 
 @pytest.mark.parametrize("dtype,shape,path", [
-    ("f32", (1, 2, 16, 15), "pair"), ("bf16", (2, 3, 74, 74), "dir-shared"),
+    ("f32", (1, 2, 16, 15), "pair"), ("bf16", (2, 3, 74, 74), "dir-half"),
+    ("bf16", (2, 3, 21, 2), "dir-shared"), ("bf16", (2, 3, 21, 4), "dir-half"),
     ("f32", (1, 2, 16, 15), "split"), ("bf16", (2, 3, 74, 74), "split"),
     ("f32", (1, 2, 60, 100), "split"),
     ("f32", (1, 2, 37, 38), "dir"), ("f32", (1, 2, 19, 150), "dir"),
-    ("bf16", (1, 2, 148, 148), "dir-shared"), ("f32", (1, 1, 256, 256), "dir-yglobal"),
+    ("bf16", (1, 2, 148, 148), "dir-half"), ("f32", (1, 1, 256, 256), "dir-yglobal"),
     ("bf16", (1, 2, 19, 23), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
@@ -342,7 +345,11 @@ def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("shape,dtype,path", [
-    ((2, 3, 74, 74), "bf16", "split"),         # fewer planes than SMs
+    ((2, 3, 74, 74), "bf16", "split"),         # few planes: at most two waves of four CTAs
+    ((2, 64, 74, 74), "bf16", "split"),
+    ((4, 64, 74, 74), "bf16", "dir-half"),     # four waves
+    ((8, 32, 37, 37), "f32", "split"),
+    ((8, 64, 37, 37), "f32", "dir"),           # three waves
     ((2, 3, 74, 74), "f32", "split"),
     ((4, 4, 37, 37), "f32", "split"),
     ((1, 4, 16, 16), "f32", "split"),
@@ -350,13 +357,13 @@ def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
     ((1, 2, 20, 33), "bf16", "split"),         # odd bf16 row width
     ((8, 24, 16, 16), "f32", "pair"),          # lines of up to 16
     ((8, 24, 16, 14), "bf16", "pair"),
-    ((4, 40, 37, 37), "f32", "dir"),
-    ((4, 40, 74, 74), "bf16", "dir-shared"),
-    ((4, 40, 20, 33), "bf16", "generic"),      # odd bf16 row width
+    ((8, 40, 37, 37), "f32", "dir"),
+    ((8, 40, 74, 74), "bf16", "dir-half"),
+    ((8, 40, 20, 33), "bf16", "generic"),      # odd bf16 row width
     ((1, 2, 160, 160), "f32", "dir-shared"),   # lines over 128; two output planes do not fit
     ((1, 2, 256, 256), "f32", "dir-yglobal"),
     ((1, 2, 256, 256), "bf16", "dir-banded"),
-    ((1, 2, 148, 148), "bf16", "dir-shared"),
+    ((1, 2, 148, 148), "bf16", "dir-half"),
     ((1, 1, 300, 40), "f32", "generic"),       # line longer than 256
     ((2, 2, 1, 40), "bf16", "generic"),        # lines of one position
     ((1, 3, 17, 1), "f32", "generic"),
@@ -439,9 +446,9 @@ def test_output_fully_overwritten(gspn):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dtype,shape,path", [
-    ("bf16", (2, 4, 74, 74), "dir-shared"), ("f32", (1, 6, 16, 16), "pair"),
+    ("bf16", (2, 4, 74, 74), "dir-half"), ("f32", (1, 6, 16, 16), "pair"),
     ("bf16", (2, 4, 74, 74), "split"), ("f32", (1, 4, 37, 38), "split"),
-    ("f32", (1, 4, 19, 150), "dir"), ("bf16", (1, 4, 19, 150), "dir-shared"),
+    ("f32", (1, 4, 19, 150), "dir"), ("bf16", (1, 4, 19, 150), "dir-half"),
     ("bf16", (1, 4, 20, 33), "generic")],
     ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
 @pytest.mark.parametrize("gate_dirs,groups", [(1, "all"), (4, "half"), (1, "one"), (4, "one")])
