@@ -341,7 +341,8 @@ struct RowScan {
     // raw buffers are indexed statically.  Three lines while a line's words
     // fit 18 registers, fewer for longer lines so that the lookahead stays
     // within about 54 registers (beyond that the kernel spills).
-    static constexpr int kDepth = kTensors * kWords <= 18 ? 3 : kTensors * kWords <= 24 ? 2 : 1;
+    static constexpr int kDepth = kTensors * kWords <= 18 ? (es == 2 && kTensors * kWords <= 12 ? 4 : 3)
+                                  : kTensors * kWords <= 24 ? 2 : 1;
     static constexpr int kUnroll = kDepth % 2 == 0 ? kDepth : 2 * kDepth;
     static constexpr int kPrefetchAhead = 8;    // lines between an L2 prefetch and its use
     static constexpr int kPrefetchLines = kUnroll;   // lines per prefetch (one per loop body)
