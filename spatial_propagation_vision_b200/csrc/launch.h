@@ -23,7 +23,7 @@ struct LaunchInfo {
 };
 
 struct DeviceProps {
-    int sms = 0, smem_optin = 0, smem_per_sm = 0, major = 0, minor = 0;
+    int sms = 0, smem_optin = 0, smem_per_sm = 0, major = 0, minor = 0, l2_bytes = 0;
 };
 
 // Launch geometry of the direction kernel.
@@ -64,7 +64,8 @@ cudaError_t launch_pair_f32(int RP, int NS, const gspn::PairParams &pp, int smem
 cudaError_t kernel_occupancy(const void *kernel, int threads, int smem, int &per_sm);
 
 // Backward kernel (fp32 gradients); the caller zeroed the gradient buffers.
-cudaError_t launch_bwd(const gspn::BwdParams &bp, bool bf16, int smem, const DeviceProps &dp,
+// `cap` > 0 limits the resident CTAs per SM.
+cudaError_t launch_bwd(const gspn::BwdParams &bp, bool bf16, int smem, const DeviceProps &dp, int cap,
                        cudaStream_t s, LaunchInfo &li);
 
 // Normalised weights of the compact mode into the workspace (one launch).
