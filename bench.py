@@ -46,16 +46,26 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha() -> str:
-    """sha256 over the device-side CUDA sources (sorted by name): every file
-    under csrc/ except gspn_api.cu, the host C ABI (argument checks, planner).
-    The planner's choice is checked separately: a profile also records the
-    launch geometry it was taken with."""
+# The translation units that instantiate each kernel (its device code also
+# comes from every header under csrc/).
+KERNEL_UNITS = {"prop2d_dir_kernel": ("dir_",), "prop2d_pair_kernel": ("pair_",),
+                "prop2d_split_kernel": ("split_",), "prop2d_generic_kernel": ("generic_",),
+                "prop2d_norm_kernel": ("norm_",), "prop2d_bwd_kernel": ("bwd_",)}
+
+
+def kernel_sources_sha(kernel: str = "prop2d_dir_kernel") -> str:
+    """sha256 over the sources of one kernel's device code, sorted by name:
+    every header (`.cuh`) under csrc/ and the kernel's own translation units
+    (KERNEL_UNITS). Host-only files (the C ABI, launch.h, other kernels'
+    launchers) are left out, so they can change without invalidating a
+    profile; the planner's choice is checked separately, since a profile also
+    records the launch geometry it was taken with."""
     import glob
     import hashlib
     h = hashlib.sha256()
+    units = KERNEL_UNITS.get(kernel, ())
     files = sorted(f for f in glob.glob(os.path.join(ROOT, "spatial_propagation_vision_b200", "csrc", "*"))
-                   if os.path.basename(f) != "gspn_api.cu")
+                   if f.endswith(".cuh") or (f.endswith(".cu") and os.path.basename(f).startswith(units)))
     for f in files:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
@@ -84,7 +94,7 @@ def profiled_traffic(kernel: str, workload: str, launch: dict | None = None):
     text = open(path).read()
     sha = re.search(r"kernel_sources_sha256:\s*([0-9a-f]{64})", text)
     tb = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    if not sha or not tb or sha.group(1) != kernel_sources_sha():
+    if not sha or not tb or sha.group(1) != kernel_sources_sha(kernel):
         return None
     if launch is not None:
         geo = re.search(r"launch_geometry:\s*grid=(\d+)\s+block=(\d+)\s+smem=(\d+)", text)

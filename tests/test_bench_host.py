@@ -81,13 +81,13 @@ def test_reference_arm_other_ranks_are_silent(capsys, monkeypatch):
 @pytest.mark.parametrize("matches", [True, False])
 def test_profile_traffic_needs_current_sources(tmp_path, monkeypatch, matches):
     os.makedirs(tmp_path / "profiles")
-    sha = bench.kernel_sources_sha() if matches else "0" * 64
+    sha = bench.kernel_sources_sha("prop2d_pair_kernel") if matches else "0" * 64
     (tmp_path / "profiles" / "prop2d_pair_1k.md").write_text(
         f"kernel_sources_sha256: {sha}\ntraffic_bytes_per_launch: 12345\n"
         "launch_geometry: grid=444 block=128 smem=53552\n")
-    real_sha = bench.kernel_sources_sha()
+    real_sha = {k: bench.kernel_sources_sha(k) for k in bench.KERNEL_UNITS}
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_sources_sha", lambda: real_sha)
+    monkeypatch.setattr(bench, "kernel_sources_sha", lambda kernel="prop2d_dir_kernel": real_sha[kernel])
     assert bench.profiled_traffic("prop2d_pair_kernel", "1k") == (12345 if matches else None)
     assert bench.profiled_traffic("prop2d_dir_kernel", "1k") is None
     same = {"grid": 444, "block": 128, "smem": 53552}
@@ -109,3 +109,14 @@ def test_clock_summary_is_honest_about_short_windows():
     cs.t1 = 11.3
     out = cs.summary()
     assert out["source"] == "timed region" and out["samples"] == 1 and out["sm_mhz"] == 1965.0
+
+
+def test_kernel_hash_ignores_host_only_files():
+    """A kernel's source hash covers the device headers and its own units,
+    not the C ABI or another kernel's launcher."""
+    import glob
+    csrc = os.path.join(bench.ROOT, "spatial_propagation_vision_b200", "csrc")
+    names = {os.path.basename(f) for f in glob.glob(os.path.join(csrc, "*"))}
+    assert "gspn_api.cu" in names and "launch.h" in names and "bwd_launch.cu" in names
+    shas = {k: bench.kernel_sources_sha(k) for k in bench.KERNEL_UNITS}
+    assert len(set(shas.values())) == len(shas)     # every kernel has its own units
