@@ -54,22 +54,26 @@ KERNEL_UNITS = {"prop2d_dir_kernel": ("dir_",), "prop2d_pair_kernel": ("pair_",)
 
 
 def kernel_sources_sha(kernel: str = "prop2d_dir_kernel") -> str:
-    """sha256 over the sources of one kernel's device code, sorted by name:
-    every header (`.cuh`) under csrc/ and the kernel's own translation units
-    (KERNEL_UNITS). Host-only files (the C ABI, launch.h, other kernels'
+    """sha256 over the code (comments and blank lines left out) of one
+    kernel's device sources, sorted by name: every header (`.cuh`) under
+    csrc/ and the kernel's own translation units (KERNEL_UNITS). Host-only files (the C ABI, launch.h, other kernels'
     launchers) are left out, so they can change without invalidating a
     profile; the planner's choice is checked separately, since a profile also
     records the launch geometry it was taken with."""
     import glob
     import hashlib
+    import re
     h = hashlib.sha256()
     units = KERNEL_UNITS.get(kernel, ())
     files = sorted(f for f in glob.glob(os.path.join(ROOT, "spatial_propagation_vision_b200", "csrc", "*"))
                    if f.endswith(".cuh") or (f.endswith(".cu") and os.path.basename(f).startswith(units)))
+    # comments and blank lines do not change the code: they are left out
+    strip = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
     for f in files:
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            code = strip.sub("", fh.read())
+        h.update("\n".join(ln.rstrip() for ln in code.splitlines() if ln.strip()).encode())
     return h.hexdigest()
 
 

@@ -26,9 +26,10 @@
 //
 // Input staging:
 //   * row lines: each lane loads its words of a line straight from global
-//     memory (read-only path), three lines ahead into registers; one lane
-//     per tensor issues a bulk L2 prefetch (TMA engine) of the lines about
-//     to be read, eight lines ahead, continuing into the warp's next plane;
+//     memory (read-only path), three or four lines ahead into registers; one
+//     lane per tensor issues a bulk L2 prefetch (TMA engine) of the lines
+//     about to be read, eight lines ahead, continuing into the warp's next
+//     plane;
 //   * column lines: a chunk is a strip of 16 bytes of every grid row (8 bf16
 //     or 4 fp32 columns), copied by the warp with 4-byte cp.async (four lanes
 //     per grid row) into a two-stage ring.  The strip rows of the six tensors
@@ -36,12 +37,13 @@
 //     words of a strip row in reverse order, so both sweeps meet their
 //     columns in scan order.  A four-step body reads its columns with one
 //     8-byte read per tensor and position (bf16; two for fp32).
-// Outputs u * h are accumulated in fp32 in shared memory and written once,
-// converted, at the end of the plane (modes below): one plane that all
-// directions add into with shared-memory atomics, or two planes (rows,
+// Outputs u * h are accumulated in shared memory and written once,
+// converted, at the end of the plane (modes below): two planes (rows,
 // columns) written without atomics, each shared by a sweep pair that splits
-// at the midpoint; global atomics and row bands cover planes too large for
-// shared memory.
+// at the midpoint (fp32 planes, or for bf16 inputs bf16 planes of pair words
+// whose column midpoint is word-aligned); one fp32 plane that all directions
+// add into with shared-memory atomics; global atomics and row bands cover
+// planes too large for shared memory.
 //
 // Positions past the end of a line (q >= M) compute finite garbage that
 // never reaches a valid position: their right-hand neighbour term of
