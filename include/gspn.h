@@ -206,7 +206,10 @@ gspn_status gspn_prop2d_fwd_ws(const void *x, const void *lambda, const void *wl
  * caller's device buffers (d_x, d_lambda, d_wlogit, d_u), runs
  * gspn_prop2d_fwd into d_out and copies d_out back into h_out, in up to four
  * batch chunks whose uploads, kernels and downloads overlap (chunk k+1 is
- * uploaded while chunk k runs and chunk k-1 comes back).  The chunks run on
+ * uploaded while chunk k runs and chunk k-1 comes back).  A chunk starts at
+ * a batch index whose byte offset is a multiple of 16 in every tensor, so
+ * that the kernels' alignment rule holds for every chunk (one chunk when no
+ * such split exists).  The chunks run on
  * three streams and a few events that the library creates once per device
  * (no device memory); they start after the work already queued on `stream`.
  * Returns after everything has finished, so h_out is valid on return.

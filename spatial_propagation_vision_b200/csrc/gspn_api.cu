@@ -554,12 +554,24 @@ extern "C" gspn_status gspn_prop2d_fwd_host(const void *h_x, const void *h_lambd
     // the pipeline starts after the work already queued on `stream`
     if (cudaEventRecord(hp->start, stream) != cudaSuccess) return GSPN_ERR_CUDA;
     if (cudaStreamWaitEvent(hp->up, hp->start, 0) != cudaSuccess) return GSPN_ERR_CUDA;
-    const int nchunk = B < kHostChunks ? B : kHostChunks;
+    // Chunks start at multiples of m batch elements, m the least count whose
+    // bytes in every tensor are a multiple of 16, so that each chunk's device
+    // pointers keep the kernels' 16-byte alignment.
+    auto lcm16 = [](size_t bytes) { size_t m = 1; while ((m * bytes) % 16) ++m; return m; };
+    const size_t mx_ = lcm16(bx), mw_ = lcm16(bw);
+    size_t m = mx_;
+    while (m % mw_) m += mx_;
+    const long long units = (static_cast<long long>(B) + static_cast<long long>(m) - 1) / static_cast<long long>(m);
+    const int nchunk = units < kHostChunks ? static_cast<int>(units) : kHostChunks;
     auto cb = [](const void *p, size_t off) { return static_cast<const char *>(p) + off; };
     auto mb = [](void *p, size_t off) { return static_cast<char *>(p) + off; };
+    auto edge = [&](int c) {
+        const long long b = static_cast<long long>(m) * (units * c / nchunk);
+        return static_cast<int>(b < B ? b : B);
+    };
     for (int c = 0; c < nchunk; ++c) {
-        const int b0 = static_cast<int>(static_cast<long long>(B) * c / nchunk);
-        const int b1 = static_cast<int>(static_cast<long long>(B) * (c + 1) / nchunk);
+        const int b0 = edge(c);
+        const int b1 = edge(c + 1);
         const size_t n = static_cast<size_t>(b1 - b0);
         if (cudaMemcpyAsync(mb(d_x, b0 * bx), cb(h_x, b0 * bx), n * bx, cudaMemcpyHostToDevice, hp->up) ||
             cudaMemcpyAsync(mb(d_lambda, b0 * bg), cb(h_lambda, b0 * bg), n * bg, cudaMemcpyHostToDevice, hp->up) ||

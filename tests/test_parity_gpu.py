@@ -398,8 +398,15 @@ def test_algo_refused_when_out_of_range(gspn, shape, dtype, algo):
     assert bool((out == 7.0).all())
 
 
-def test_host_entry_point(gspn):
-    inp = make_inputs(2, 3, 37, 40, sigma_w=2.0, dtype="bf16", seed=4)
+@pytest.mark.parametrize("shape,dtype", [((2, 3, 37, 40), "bf16"), ((1, 1, 5, 5), "f32"),
+                                         ((5, 1, 5, 5), "f32"), ((7, 2, 9, 6), "bf16"),
+                                         ((3, 1, 3, 3), "bf16")],
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_host_entry_point(gspn, shape, dtype):
+    """Pipelined batch chunks, also when a batch element's bytes are not a
+    multiple of 16 (chunks then start at aligned batch indices)."""
+    B, Cc, H, W = shape
+    inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=4)
     h = {k: v.pin_memory() for k, v in inp.items()}
     h["out"] = torch.empty_like(inp["x"]).pin_memory()
     d = {k: torch.empty_like(v, device="cuda") for k, v in h.items()}
@@ -409,8 +416,9 @@ def test_host_entry_point(gspn):
     torch.cuda.synchronize()
     yo = oracle.prop2d(f64(inp["x"]), f64(inp["lam"]), f64(inp["wlogit"]), f64(inp["u"]))
     scale = np.max(np.abs(yo))
-    assert np.max(np.abs(f64(y) - yo)) <= 2e-2 * scale
-    assert np.max(np.abs(f64(y) - f64(y_dev))) <= 1e-2 * scale
+    tol = TOL[inp["x"].dtype]
+    assert np.max(np.abs(f64(y) - yo)) <= tol * scale
+    assert np.max(np.abs(f64(y) - f64(y_dev))) <= tol * scale
 
 
 def test_side_stream(gspn):
