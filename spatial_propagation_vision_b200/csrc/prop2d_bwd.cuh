@@ -22,7 +22,9 @@
 // segment of kSeg lines from its checkpoint into a segment buffer and walks
 // it backwards.  Shared memory per warp: (L / kSeg + kSeg + 1) lines.
 // Weights are recomputed in the plain form (sigmoid, local sum, clamp,
-// divide) in fp32 in both sweeps.  Gradients are fp32: dlambda, du and (per
+// divide) in fp32 in both sweeps.  Every sweep loads the next line's inputs
+// one step ahead, into registers, so that a step does not wait for its own
+// loads.  Gradients are fp32: dlambda, du and (per
 // channel) dwlogit are stored once; dx adds the four directions with global
 // fp32 atomics, and shared logit fields (share_w) add over the channels
 // likewise, into buffers the host zeroed.
@@ -58,6 +60,13 @@ __device__ __forceinline__ float bwd_sigmoid(float z) {
     return rcp(1.0f + ex2(z * -1.4426950408889634f));
 }
 
+// Inputs of a lane's R positions of one line: the three logit slots,
+// lambda, x, and (reverse sweep) u and the output gradient.
+template <int R>
+struct BwdIn {
+    float z[3][R], lam[R], x[R], u[R], gy[R];
+};
+
 template <typename T, int R>
 struct BwdLine {
     const BwdParams &p;
@@ -92,23 +101,44 @@ struct BwdLine {
         return rows ? static_cast<size_t>(line) * p.W + q : static_cast<size_t>(q) * p.W + line;
     }
 
-    // normalised weights (w), sigmoids (s) and local sum (S) of position q
-    __device__ __forceinline__ void weights(size_t e, int q, float (&s)[3], float (&w)[3], float &S) const {
+    // Inputs of line s (positions past the line's end read position M-1:
+    // finite, never used; off-grid logit slots are read but never used).
+    template <bool REV>
+    __device__ __forceinline__ void load_in(int s, BwdIn<R> &in) const {
         const size_t HW = static_cast<size_t>(p.H) * p.W;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = min(lane * R + r, M - 1);
+            const size_t e = idx(s, q);
+#pragma unroll
+            for (int k = 0; k < 3; ++k) in.z[k][r] = bwd_in(wl, k * HW + e);
+            in.lam[r] = bwd_in(lam, e);
+            in.x[r] = bwd_in(x, e);
+            if (REV) {
+                in.u[r] = bwd_in(u, e);
+                in.gy[r] = bwd_in(gy, e);
+            }
+        }
+    }
+
+    // normalised weights (w), sigmoids (s) and local sum (S) of position
+    // q = lane R + r; off-grid slots are selected away
+    __device__ __forceinline__ void weights(const BwdIn<R> &in, int r, int q, float (&s)[3], float (&w)[3],
+                                            float &S) const {
         S = 0.f;
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int nb = q + k - 1;
-            s[k] = (nb >= 0 && nb < M) ? bwd_sigmoid(bwd_in(wl, k * HW + e)) : 0.f;
+            s[k] = (nb >= 0 && nb < M) ? bwd_sigmoid(in.z[k][r]) : 0.f;
             S += s[k];
         }
-        const float r = 1.0f / fmaxf(S, 1e-6f);
+        const float rs = 1.0f / fmaxf(S, 1e-6f);
 #pragma unroll
-        for (int k = 0; k < 3; ++k) w[k] = s[k] * r;
+        for (int k = 0; k < 3; ++k) w[k] = s[k] * rs;
     }
 
     // one forward step: h <- W h + lambda x (positions past the end stay 0)
-    __device__ __forceinline__ void fwd_step(int s, float (&h)[R]) const {
+    __device__ __forceinline__ void fwd_step(const BwdIn<R> &in, float (&h)[R]) const {
         const float hl = __shfl_up_sync(0xffffffffu, h[R - 1], 1);
         const float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
         float hn[R];
@@ -116,15 +146,32 @@ struct BwdLine {
         for (int r = 0; r < R; ++r) {
             const int q = lane * R + r;
             if (q >= M) { hn[r] = 0.f; continue; }
-            const size_t e = idx(s, q);
             float sg[3], w[3], S;
-            weights(e, q, sg, w, S);
+            weights(in, r, q, sg, w, S);
             const float left = r > 0 ? h[r > 0 ? r - 1 : 0] : (lane > 0 ? hl : 0.f);
             const float right = r + 1 < R ? h[r + 1 < R ? r + 1 : r] : hr;
-            hn[r] = w[0] * left + w[1] * h[r] + w[2] * right + bwd_in(lam, e) * bwd_in(x, e);
+            hn[r] = w[0] * left + w[1] * h[r] + w[2] * right + in.lam[r] * in.x[r];
         }
 #pragma unroll
         for (int r = 0; r < R; ++r) h[r] = hn[r];
+    }
+
+    // steps [s0, s1) forwards from h, storing h after step s into
+    // out(s) when out is given; the next line's inputs load one step ahead
+    template <typename Out>
+    __device__ __forceinline__ void sweep(int s0, int s1, float (&h)[R], Out out) const {
+        BwdIn<R> a, b;
+        load_in<false>(s0, a);
+        for (int s = s0; s < s1; s += 2) {
+            if (s + 1 < s1) load_in<false>(s + 1, b);
+            fwd_step(a, h);
+            out(s, h);
+            if (s + 1 < s1) {
+                if (s + 2 < s1) load_in<false>(s + 2, a);
+                fwd_step(b, h);
+                out(s + 1, h);
+            }
+        }
     }
 
     __device__ __forceinline__ void store_line(float *buf, const float (&h)[R]) const {
@@ -139,16 +186,71 @@ struct BwdLine {
     // The whole backward of this direction.  `ck`: checkpoint lines
     // (line i holds h after step i * kSeg + kSeg - 1), `seg`: kSeg + 1 lines
     // (line 0: h before the segment, line 1 + t: after its step t).
+    // The reverse step s (adjoint of line s): gradients of line s's inputs,
+    // the carry into line s-1.  hcur / hprv: h after steps s and s-1.
+    __device__ __forceinline__ void rev_step(int s, const BwdIn<R> &in, const float *hcur, const float *hprv,
+                                             float (&carry)[R]) const {
+        const size_t HW = static_cast<size_t>(p.H) * p.W;
+        float cl = 0.f, cr = 0.f, cmid[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) cmid[r] = 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = lane * R + r;
+            if (q >= M) continue;
+            const size_t e = idx(s, q);
+            const float gyv = in.gy[r];
+            const float a = in.u[r] * gyv + carry[r];
+            du[e] = gyv * hcur[q];
+            dlam[e] = a * in.x[r];
+            atomicAdd(dx + e, a * in.lam[r]);
+            float sgm[3], w[3], S;
+            weights(in, r, q, sgm, w, S);
+            float dw[3], dot = 0.f;
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const int nb = q + k - 1;
+                dw[k] = (nb >= 0 && nb < M && s > 0) ? a * hprv[nb] : 0.f;
+                dot += dw[k] * w[k];
+            }
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const int nb = q + k - 1;
+                if (nb < 0 || nb >= M) continue;
+                const float ds = S > 1e-6f ? (dw[k] - dot) / S : dw[k] * 1e6f;
+                const float dz = ds * sgm[k] * (1.f - sgm[k]);
+                if (p.share_w) atomicAdd(dwl + k * HW + e, dz);
+                else dwl[k * HW + e] = dz;
+            }
+            // transposed stencil: position q passes w_k a to q + k - 1
+            const float c0 = w[0] * a, c1 = w[1] * a, c2 = w[2] * a;
+            cmid[r] += c1;
+            if (r > 0) cmid[r - 1 > 0 ? r - 1 : 0] += c0;
+            else cl = c0;
+            if (r + 1 < R) cmid[r + 1 < R ? r + 1 : r] += c2;
+            else cr = c2;
+        }
+        // contributions that cross lanes
+        const float from_right = __shfl_down_sync(0xffffffffu, cl, 1);   // lane+1's position 0 -> my last
+        const float from_left = __shfl_up_sync(0xffffffffu, cr, 1);      // lane-1's last -> my first
+#pragma unroll
+        for (int r = 0; r < R; ++r) carry[r] = cmid[r];
+        if (lane < 31) carry[R - 1] += from_right;
+        if (lane > 0) carry[0] += from_left;
+    }
+
+    // The whole backward of this direction.  `ck`: checkpoint lines
+    // (line i holds h after step i * kSeg + kSeg - 1), `seg`: kSeg + 1 lines
+    // (line 0: h before the segment, line 1 + t: after its step t).
     __device__ void run(float *ck, float *seg) const {
         const int line_f = 32 * R;
         float h[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) h[r] = 0.f;
         // forward sweep: checkpoints at the end of every segment
-        for (int s = 0; s < L; ++s) {
-            fwd_step(s, h);
-            if (s % kBwdSeg == kBwdSeg - 1) store_line(ck + (s / kBwdSeg) * line_f, h);
-        }
+        sweep(0, L, h, [&](int s, const float (&hh)[R]) {
+            if (s % kBwdSeg == kBwdSeg - 1) store_line(ck + (s / kBwdSeg) * line_f, hh);
+        });
         __syncwarp();
         float carry[R];
 #pragma unroll
@@ -164,66 +266,19 @@ struct BwdLine {
                 load_line(ck + (sg - 1) * line_f, h);
             }
             store_line(seg, h);
-            for (int s = s0; s < s1; ++s) {
-                fwd_step(s, h);
-                store_line(seg + (s - s0 + 1) * line_f, h);
-            }
+            sweep(s0, s1, h, [&](int s, const float (&hh)[R]) { store_line(seg + (s - s0 + 1) * line_f, hh); });
             __syncwarp();
-            // reverse steps of the segment
-            for (int s = s1 - 1; s >= s0; --s) {
-                const float *hcur = seg + (s - s0 + 1) * line_f;
-                const float *hprv = seg + (s - s0) * line_f;
-                float adj[R], cl = 0.f, cr = 0.f, cmid[R];
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    adj[r] = 0.f;
-                    cmid[r] = 0.f;
+            // reverse steps of the segment, the inputs of line s-1 loaded
+            // while line s is processed
+            BwdIn<R> a, b;
+            load_in<true>(s1 - 1, a);
+            for (int s = s1 - 1; s >= s0; s -= 2) {
+                if (s - 1 >= s0) load_in<true>(s - 1, b);
+                rev_step(s, a, seg + (s - s0 + 1) * line_f, seg + (s - s0) * line_f, carry);
+                if (s - 1 >= s0) {
+                    if (s - 2 >= s0) load_in<true>(s - 2, a);
+                    rev_step(s - 1, b, seg + (s - s0) * line_f, seg + (s - 1 - s0) * line_f, carry);
                 }
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int q = lane * R + r;
-                    if (q >= M) continue;
-                    const size_t e = idx(s, q);
-                    const float gyv = bwd_in(gy, e);
-                    const float a = bwd_in(u, e) * gyv + carry[r];
-                    adj[r] = a;
-                    du[e] = gyv * hcur[q];
-                    dlam[e] = a * bwd_in(x, e);
-                    atomicAdd(dx + e, a * bwd_in(lam, e));
-                    float sgm[3], w[3], S;
-                    weights(e, q, sgm, w, S);
-                    float dw[3], dot = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 3; ++k) {
-                        const int nb = q + k - 1;
-                        dw[k] = (nb >= 0 && nb < M && s > 0) ? a * hprv[nb] : 0.f;
-                        dot += dw[k] * w[k];
-                    }
-                    const size_t HW = static_cast<size_t>(p.H) * p.W;
-#pragma unroll
-                    for (int k = 0; k < 3; ++k) {
-                        const int nb = q + k - 1;
-                        if (nb < 0 || nb >= M) continue;
-                        const float ds = S > 1e-6f ? (dw[k] - dot) / S : dw[k] * 1e6f;
-                        const float dz = ds * sgm[k] * (1.f - sgm[k]);
-                        if (p.share_w) atomicAdd(dwl + k * HW + e, dz);
-                        else dwl[k * HW + e] = dz;
-                    }
-                    // transposed stencil: position q passes w_k a to q + k - 1
-                    const float c0 = w[0] * a, c1 = w[1] * a, c2 = w[2] * a;
-                    cmid[r] += c1;
-                    if (r > 0) cmid[r - 1 > 0 ? r - 1 : 0] += c0;
-                    else cl = c0;
-                    if (r + 1 < R) cmid[r + 1 < R ? r + 1 : r] += c2;
-                    else cr = c2;
-                }
-                // contributions that cross lanes
-                const float from_right = __shfl_down_sync(0xffffffffu, cl, 1);   // lane+1's position 0 -> my last
-                const float from_left = __shfl_up_sync(0xffffffffu, cr, 1);      // lane-1's last -> my first
-#pragma unroll
-                for (int r = 0; r < R; ++r) carry[r] = cmid[r];
-                if (lane < 31) carry[R - 1] += from_right;
-                if (lane > 0) carry[0] += from_left;
             }
             __syncwarp();
         }
