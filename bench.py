@@ -46,17 +46,22 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-# The translation units that instantiate each kernel (its device code also
-# comes from every header under csrc/).
-KERNEL_UNITS = {"prop2d_dir_kernel": ("dir_",), "prop2d_pair_kernel": ("pair_",),
-                "prop2d_split_kernel": ("split_",), "prop2d_generic_kernel": ("generic_",),
-                "prop2d_norm_kernel": ("norm_",), "prop2d_bwd_kernel": ("bwd_",)}
+# The sources of each kernel's device code: the headers that define it and
+# the translation units (and their launch headers) that instantiate it.
+KERNEL_UNITS = {
+    "prop2d_dir_kernel": ("device_common.cuh", "prop2d_dir.cuh", "dir_"),
+    "prop2d_pair_kernel": ("device_common.cuh", "prop2d_pair.cuh", "pair_"),
+    "prop2d_split_kernel": ("device_common.cuh", "prop2d_dir.cuh", "prop2d_split.cuh", "split_"),
+    "prop2d_generic_kernel": ("device_common.cuh", "prop2d_generic.cuh", "generic_"),
+    "prop2d_norm_kernel": ("device_common.cuh", "prop2d_norm.cuh", "norm_"),
+    "prop2d_bwd_kernel": ("device_common.cuh", "prop2d_bwd.cuh", "bwd_"),
+}
 
 
 def kernel_sources_sha(kernel: str = "prop2d_dir_kernel") -> str:
     """sha256 over the code (comments and blank lines left out) of one
-    kernel's device sources, sorted by name: every header (`.cuh`) under
-    csrc/ and the kernel's own translation units (KERNEL_UNITS). Host-only files (the C ABI, launch.h, other kernels'
+    kernel's device sources, sorted by name: the files under csrc/ whose
+    names start with one of the kernel's KERNEL_UNITS entries. Host-only files (the C ABI, launch.h, other kernels'
     launchers) are left out, so they can change without invalidating a
     profile; the planner's choice is checked separately, since a profile also
     records the launch geometry it was taken with."""
@@ -66,7 +71,7 @@ def kernel_sources_sha(kernel: str = "prop2d_dir_kernel") -> str:
     h = hashlib.sha256()
     units = KERNEL_UNITS.get(kernel, ())
     files = sorted(f for f in glob.glob(os.path.join(ROOT, "spatial_propagation_vision_b200", "csrc", "*"))
-                   if f.endswith(".cuh") or (f.endswith(".cu") and os.path.basename(f).startswith(units)))
+                   if os.path.basename(f).startswith(units))
     # comments and blank lines do not change the code: they are left out
     strip = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
     for f in files:

@@ -112,8 +112,8 @@ def test_clock_summary_is_honest_about_short_windows():
 
 
 def test_kernel_hash_ignores_host_only_files():
-    """A kernel's source hash covers the device headers and its own units,
-    not the C ABI or another kernel's launcher."""
+    """A kernel's source hash covers its own headers and units, not the C ABI
+    or another kernel's sources."""
     import glob
     csrc = os.path.join(bench.ROOT, "spatial_propagation_vision_b200", "csrc")
     names = {os.path.basename(f) for f in glob.glob(os.path.join(csrc, "*"))}
