@@ -62,6 +62,8 @@ class Oracle:
         lib.oracle_prop2d_bwd_f64.restype = ctypes.c_int
         lib.oracle_prop2d_ex_f64.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 7 + [dp]
         lib.oracle_prop2d_ex_f64.restype = ctypes.c_int
+        lib.oracle_prop2d_bwd_ex_f64.argtypes = [dp] * 5 + [ctypes.c_int] * 7 + [dp] * 4
+        lib.oracle_prop2d_bwd_ex_f64.restype = ctypes.c_int
         self._lib = lib
 
     def prop2d(self, x, lam, wlogit, u, dirs: int = 15, share_w: int = 0) -> np.ndarray:
@@ -118,6 +120,26 @@ class Oracle:
             raise ValueError("oracle_prop2d_bwd_f64 rejected its arguments")
         return g
 
+    def prop2d_bwd_ex(self, x, lam, wlogit, u, gy, dirs: int = 15, gate_dirs: int = 4,
+                      w_groups=None) -> dict:
+        """Backward of the sharing variants in fp64 (layouts of prop2d_ex): the
+        gradients {"x", "lam", "wlogit", "u"}; a shared input's gradient sums
+        the gradients of its uses."""
+        x, lam, wlogit, u, gy = (_f64(t) for t in (x, lam, wlogit, u, gy))
+        B, Cc, H, W = x.shape
+        G = Cc if w_groups is None else int(w_groups)
+        assert lam.shape == (B, gate_dirs, Cc, H, W) and u.shape == lam.shape, (lam.shape, u.shape)
+        assert wlogit.shape == (B, 4, G, 3, H, W), wlogit.shape
+        assert gy.shape == x.shape, gy.shape
+        g = {"x": np.zeros_like(x), "lam": np.zeros_like(lam), "wlogit": np.zeros_like(wlogit),
+             "u": np.zeros_like(u)}
+        rc = self._lib.oracle_prop2d_bwd_ex_f64(
+            _ptr(x), _ptr(lam), _ptr(wlogit), _ptr(u), _ptr(gy), B, Cc, H, W, int(dirs),
+            int(gate_dirs), G, _ptr(g["x"]), _ptr(g["lam"]), _ptr(g["wlogit"]), _ptr(g["u"]))
+        if rc != 0:
+            raise ValueError("oracle_prop2d_bwd_ex_f64 rejected its arguments")
+        return g
+
     def weights(self, wlogit) -> np.ndarray:
         """Normalised tridiagonal weights [B,4,Cw,3,H,W] of a logit field (0 in off-grid slots)."""
         wlogit = _f64(wlogit)
@@ -153,3 +175,8 @@ def prop2d_bwd(x, lam, wlogit, u, gy, dirs: int = 15, share_w: int = 0) -> dict:
 
 def prop2d_ex(x, lam, wlogit, u, dirs: int = 15, gate_dirs: int = 4, w_groups=None) -> np.ndarray:
     return default().prop2d_ex(x, lam, wlogit, u, dirs=dirs, gate_dirs=gate_dirs, w_groups=w_groups)
+
+
+def prop2d_bwd_ex(x, lam, wlogit, u, gy, dirs: int = 15, gate_dirs: int = 4, w_groups=None) -> dict:
+    return default().prop2d_bwd_ex(x, lam, wlogit, u, gy, dirs=dirs, gate_dirs=gate_dirs,
+                                   w_groups=w_groups)

@@ -231,19 +231,24 @@ static void position_weights(const double *wlogit, size_t wplane, int H, int W, 
     normalise_parts(lg, on, s, w, sum);
 }
 
-int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *wlogit,
-                          const double *u, const double *gy, int B, int Cc, int H, int W,
-                          int dirs, int share_w, double *dx, double *dlambda, double *dwlogit,
-                          double *du) {
+/* The backward with the sharing of the variants: lambda, u
+ * [B][gate_dirs][Cc][H][W] (gate_dirs 4, or 1 plane shared by the four
+ * directions) and logits [B][4][G][3][H][W] (channel c uses field c / (Cc/G)).
+ * A shared input's gradient is the sum of the gradients of its uses. */
+static int prop2d_bwd_shared(const double *x, const double *lambda, const double *wlogit,
+                             const double *u, const double *gy, int B, int Cc, int H, int W,
+                             int dirs, int gate_dirs, int G, double *dx, double *dlambda,
+                             double *dwlogit, double *du) {
     if (!x || !lambda || !wlogit || !u || !gy || !dx || !dlambda || !dwlogit || !du) return 1;
     if (B < 0 || Cc < 0 || H < 0 || W < 0) return 1;
     if (dirs < 1 || dirs > 15) return 1;
-    int Cw = share_w ? 1 : Cc;
+    if ((gate_dirs != 1 && gate_dirs != 4) || G < 1 || (Cc > 0 && Cc % G != 0)) return 1;
+    int cpg = Cc > 0 ? Cc / G : 1;   /* channels per logit field */
     size_t HW = (size_t)H * (size_t)W;
     memset(dx, 0, (size_t)B * (size_t)Cc * HW * sizeof(double));
-    memset(dlambda, 0, (size_t)B * 4 * (size_t)Cc * HW * sizeof(double));
-    memset(du, 0, (size_t)B * 4 * (size_t)Cc * HW * sizeof(double));
-    memset(dwlogit, 0, (size_t)B * 4 * (size_t)Cw * 3 * HW * sizeof(double));
+    memset(dlambda, 0, (size_t)B * (size_t)gate_dirs * (size_t)Cc * HW * sizeof(double));
+    memset(du, 0, (size_t)B * (size_t)gate_dirs * (size_t)Cc * HW * sizeof(double));
+    memset(dwlogit, 0, (size_t)B * 4 * (size_t)G * 3 * HW * sizeof(double));
     int maxM = H > W ? H : W;
     /* forward lines in scan order, the adjoint line and its carry */
     double *hist = (double *)calloc(HW + 1, sizeof(double));
@@ -260,9 +265,9 @@ int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *w
             size_t xpl = (size_t)b * (size_t)Cc + (size_t)c;
             for (int d = 0; d < 4; ++d) {
                 if (!(dirs & (1 << d))) continue;
-                size_t gpl = ((size_t)b * 4 + (size_t)d) * (size_t)Cc + (size_t)c;
-                size_t wpl = (((size_t)b * 4 + (size_t)d) * (size_t)Cw +
-                              (size_t)(share_w ? 0 : c)) * 3;
+                size_t gpl = ((size_t)b * (size_t)gate_dirs + (size_t)(gate_dirs == 4 ? d : 0)) *
+                             (size_t)Cc + (size_t)c;
+                size_t wpl = (((size_t)b * 4 + (size_t)d) * (size_t)G + (size_t)(c / cpg)) * 3;
                 int L = d < 2 ? H : W;
                 int M = d < 2 ? W : H;
 
@@ -295,8 +300,8 @@ int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *w
                         size_t e = at(gpl, H, W, i, j);
                         double gyv = gy[at(xpl, H, W, i, j)];
                         adj[q] = u[e] * gyv + carry[q];
-                        du[e] = gyv * hl[q];
-                        dlambda[e] = adj[q] * x[at(xpl, H, W, i, j)];
+                        du[e] += gyv * hl[q];
+                        dlambda[e] += adj[q] * x[at(xpl, H, W, i, j)];
                         dx[at(xpl, H, W, i, j)] += adj[q] * lambda[e];
                         carry_next[q] = 0.0;
                     }
@@ -327,6 +332,25 @@ int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *w
     free(carry);
     free(carry_next);
     return 0;
+}
+
+/* Backward of Prop2D: per-direction lambda, u [B][4][Cc][H][W]; logits
+ * per channel, or shared by all channels (share_w). */
+int oracle_prop2d_bwd_f64(const double *x, const double *lambda, const double *wlogit,
+                          const double *u, const double *gy, int B, int Cc, int H, int W,
+                          int dirs, int share_w, double *dx, double *dlambda, double *dwlogit,
+                          double *du) {
+    return prop2d_bwd_shared(x, lambda, wlogit, u, gy, B, Cc, H, W, dirs, 4, share_w ? 1 : (Cc > 0 ? Cc : 1),
+                             dx, dlambda, dwlogit, du);
+}
+
+/* Backward of the sharing variants (oracle_prop2d_ex_f64's layouts). */
+int oracle_prop2d_bwd_ex_f64(const double *x, const double *lambda, const double *wlogit,
+                             const double *u, const double *gy, int B, int Cc, int H, int W,
+                             int dirs, int gate_dirs, int w_groups, double *dx, double *dlambda,
+                             double *dwlogit, double *du) {
+    return prop2d_bwd_shared(x, lambda, wlogit, u, gy, B, Cc, H, W, dirs, gate_dirs, w_groups,
+                             dx, dlambda, dwlogit, du);
 }
 
 /*

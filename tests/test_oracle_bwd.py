@@ -23,10 +23,10 @@ MUTANTS = {
     # adjoint not carried to the previous line
     "no_carry": ("double *t = carry; carry = carry_next; carry_next = t;", ";"),
     # du from the adjoint instead of the output gradient
-    "du_from_adjoint": ("du[e] = gyv * hl[q];", "du[e] = adj[q] * hl[q];"),
+    "du_from_adjoint": ("du[e] += gyv * hl[q];", "du[e] += adj[q] * hl[q];"),
     # dlambda from the output gradient instead of the adjoint
-    "dlambda_from_gy": ("dlambda[e] = adj[q] * x[at(xpl, H, W, i, j)];",
-                        "dlambda[e] = gyv * x[at(xpl, H, W, i, j)];"),
+    "dlambda_from_gy": ("dlambda[e] += adj[q] * x[at(xpl, H, W, i, j)];",
+                        "dlambda[e] += gyv * x[at(xpl, H, W, i, j)];"),
     # dw taken against the current line instead of the previous one
     "dw_current_line": ("dw[k] = hprv ? adj[q] * hprv[q + k - 1] : 0.0;",
                         "dw[k] = adj[q] * hl[q + k - 1];"),
