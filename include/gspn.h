@@ -299,6 +299,25 @@ gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const void *wlogi
                             int share_w, gspn_dtype dtype, float *dx, float *dlambda,
                             float *dwlogit, float *du, cudaStream_t stream);
 
+/*
+ * gspn_prop2d_bwd_ex -- gspn_prop2d_bwd for the sharing variants of
+ * gspn_prop2d_fwd_ex (gate_dirs, w_groups as there).  A shared input's
+ * gradient is the sum of the gradients of its uses:
+ *   dlambda, du  [B][gate_dirs][Cc][H][W]  (gate_dirs = 1: summed over the
+ *                                           enabled directions)
+ *   dwlogit      [B][4][G][3][H][W]        (summed over the Cc / G channels
+ *                                           of each field)
+ *   dx           [B][Cc][H][W]
+ * Returns GSPN_ERR_SHARING for a gate_dirs other than 1 or 4 or a w_groups
+ * that does not divide Cc, before anything runs.  Other arguments and errors
+ * as gspn_prop2d_bwd; gate_dirs = 4, w_groups = Cc (or 1) is gspn_prop2d_bwd
+ * with share_w = 0 (or 1).
+ */
+gspn_status gspn_prop2d_bwd_ex(const void *x, const void *lambda, const void *wlogit,
+                               const void *u, const void *gy, int B, int Cc, int H, int W,
+                               int dirs, int gate_dirs, int w_groups, gspn_dtype dtype, float *dx,
+                               float *dlambda, float *dwlogit, float *du, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gspn_status_str(gspn_status status);
 

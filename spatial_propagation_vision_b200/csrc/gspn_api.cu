@@ -652,14 +652,14 @@ namespace {
 constexpr int kMaxBwdLine = 256;   // lines the backward kernel holds (8 positions per lane)
 }  // namespace
 
-extern "C" gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const void *wlogit,
-                                       const void *u, const void *gy, int B, int Cc, int H, int W,
-                                       int dirs, int share_w, gspn_dtype dtype, float *dx,
-                                       float *dlambda, float *dwlogit, float *du,
-                                       cudaStream_t stream) {
+namespace {
+
+gspn_status prop2d_bwd_run(const void *x, const void *lambda, const void *wlogit, const void *u,
+                           const void *gy, int B, int Cc, int H, int W, int dirs, Sharing sh,
+                           gspn_dtype dtype, float *dx, float *dlambda, float *dwlogit, float *du,
+                           cudaStream_t stream) {
     g_last = LaunchInfo{};
     if (B < 0 || Cc < 0 || H < 0 || W < 0) return GSPN_ERR_SHAPE;
-    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
     if (dtype != GSPN_F32 && dtype != GSPN_BF16) return GSPN_ERR_DTYPE;
     if (B == 0 || Cc == 0 || H == 0 || W == 0) return GSPN_OK;
     if (!x || !lambda || !wlogit || !u || !gy || !dx || !dlambda || !dwlogit || !du)
@@ -676,15 +676,18 @@ extern "C" gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const 
     if (dp.major != 10) return GSPN_ERR_DEVICE;
     const size_t plane = static_cast<size_t>(H) * W * sizeof(float);
     const size_t nx = static_cast<size_t>(B) * Cc * plane;
-    const size_t nw = static_cast<size_t>(B) * 4 * (share_w ? 1 : Cc) * 3 * plane;
+    const size_t nw = static_cast<size_t>(B) * 4 * sh.w_groups * 3 * plane;
     if (cudaMemsetAsync(dx, 0, nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemsetAsync(dlambda, 0, 4 * nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemsetAsync(du, 0, 4 * nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemsetAsync(dlambda, 0, sh.gate_dirs * nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemsetAsync(du, 0, sh.gate_dirs * nx, stream) != cudaSuccess) return GSPN_ERR_CUDA;
     if (cudaMemsetAsync(dwlogit, 0, nw, stream) != cudaSuccess) return GSPN_ERR_CUDA;
     gspn::BwdParams bp{};
     bp.x = x; bp.lam = lambda; bp.wl = wlogit; bp.u = u; bp.gy = gy;
     bp.dx = dx; bp.dlam = dlambda; bp.dwl = dwlogit; bp.du = du;
-    bp.B = B; bp.Cc = Cc; bp.H = H; bp.W = W; bp.dirs = dirs; bp.share_w = share_w;
+    bp.B = B; bp.Cc = Cc; bp.H = H; bp.W = W; bp.dirs = dirs;
+    bp.gate_dirs = sh.gate_dirs;
+    bp.w_groups = sh.w_groups;
+    bp.w_cpg = Cc / sh.w_groups;
     bp.R = (maxline + 31) / 32;
     bp.n_ckpt = (maxline + gspn::kBwdSeg - 1) / gspn::kBwdSeg;
     bp.warp_floats = (bp.n_ckpt + gspn::kBwdSeg + 1) * 32 * bp.R;
@@ -703,4 +706,31 @@ extern "C" gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const 
     const int cap = static_cast<double>(B) * Cc * per_plane > static_cast<double>(dp.l2_bytes) ? 2 : 0;
     const cudaError_t e = launch_bwd(bp, dtype == GSPN_BF16, smem, dp, cap, stream, g_last);
     return e == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" gspn_status gspn_prop2d_bwd(const void *x, const void *lambda, const void *wlogit,
+                                       const void *u, const void *gy, int B, int Cc, int H, int W,
+                                       int dirs, int share_w, gspn_dtype dtype, float *dx,
+                                       float *dlambda, float *dwlogit, float *du,
+                                       cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (dirs < 1 || dirs > 15 || (share_w != 0 && share_w != 1)) return GSPN_ERR_DIRS;
+    return prop2d_bwd_run(x, lambda, wlogit, u, gy, B, Cc, H, W, dirs,
+                          Sharing{4, share_w ? 1 : (Cc > 0 ? Cc : 1)}, dtype, dx, dlambda, dwlogit,
+                          du, stream);
+}
+
+extern "C" gspn_status gspn_prop2d_bwd_ex(const void *x, const void *lambda, const void *wlogit,
+                                          const void *u, const void *gy, int B, int Cc, int H,
+                                          int W, int dirs, int gate_dirs, int w_groups,
+                                          gspn_dtype dtype, float *dx, float *dlambda,
+                                          float *dwlogit, float *du, cudaStream_t stream) {
+    g_last = LaunchInfo{};
+    if (dirs < 1 || dirs > 15) return GSPN_ERR_DIRS;
+    if ((gate_dirs != 1 && gate_dirs != 4) || w_groups < 1 || (Cc > 0 && Cc % w_groups != 0))
+        return GSPN_ERR_SHARING;
+    return prop2d_bwd_run(x, lambda, wlogit, u, gy, B, Cc, H, W, dirs, Sharing{gate_dirs, w_groups},
+                          dtype, dx, dlambda, dwlogit, du, stream);
 }

@@ -26,7 +26,9 @@
 // one step ahead, into registers, so that a step does not wait for its own
 // loads.  Gradients are fp32: dlambda, du and (per
 // channel) dwlogit are stored once; dx adds the four directions with global
-// fp32 atomics, and shared logit fields (share_w) add over the channels
+// fp32 atomics, and shared inputs add over their uses likewise (lambda and u
+// shared by the four directions: their gradients add over the directions;
+// a logit field shared by a group of channels: over the channels)
 // likewise, into buffers the host zeroed.
 #pragma once
 
@@ -43,7 +45,9 @@ constexpr int kBwdSeg = 16;        // lines per recomputed segment
 struct BwdParams {
     const void *x, *lam, *wl, *u, *gy;
     float *dx, *dlam, *dwl, *du;
-    int B, Cc, H, W, dirs, share_w;
+    int B, Cc, H, W, dirs;
+    int gate_dirs;          // direction slots of lambda and u: 4, or 1 shared by all directions
+    int w_groups, w_cpg;    // logit fields per (batch, direction) and channels per field
     int R;            // positions per lane (line capacity 32 R >= max(H, W))
     int n_ckpt;       // checkpoint lines per warp (ceil(maxL / kBwdSeg))
     int warp_floats;  // shared-memory floats per warp
@@ -81,9 +85,8 @@ struct BwdLine {
           L(d_ < 2 ? p_.H : p_.W), M(d_ < 2 ? p_.W : p_.H) {
         const size_t HW = static_cast<size_t>(p.H) * p.W;
         const size_t xo = (static_cast<size_t>(b) * p.Cc + c) * HW;
-        const size_t go = ((static_cast<size_t>(b) * 4 + d) * p.Cc + c) * HW;
-        const int Cw = p.share_w ? 1 : p.Cc;
-        const size_t wo = (((static_cast<size_t>(b) * 4 + d) * Cw + (p.share_w ? 0 : c)) * 3) * HW;
+        const size_t go = ((static_cast<size_t>(b) * p.gate_dirs + (p.gate_dirs == 4 ? d : 0)) * p.Cc + c) * HW;
+        const size_t wo = (((static_cast<size_t>(b) * 4 + d) * p.w_groups + c / p.w_cpg) * 3) * HW;
         x = static_cast<const T *>(p.x) + xo;
         gy = static_cast<const T *>(p.gy) + xo;
         lam = static_cast<const T *>(p.lam) + go;
@@ -201,8 +204,13 @@ struct BwdLine {
             const size_t e = idx(s, q);
             const float gyv = in.gy[r];
             const float a = in.u[r] * gyv + carry[r];
-            du[e] = gyv * hcur[q];
-            dlam[e] = a * in.x[r];
+            if (p.gate_dirs == 1) {
+                atomicAdd(du + e, gyv * hcur[q]);
+                atomicAdd(dlam + e, a * in.x[r]);
+            } else {
+                du[e] = gyv * hcur[q];
+                dlam[e] = a * in.x[r];
+            }
             atomicAdd(dx + e, a * in.lam[r]);
             float sgm[3], w[3], S;
             weights(in, r, q, sgm, w, S);
@@ -219,7 +227,7 @@ struct BwdLine {
                 if (nb < 0 || nb >= M) continue;
                 const float ds = S > 1e-6f ? (dw[k] - dot) / S : dw[k] * 1e6f;
                 const float dz = ds * sgm[k] * (1.f - sgm[k]);
-                if (p.share_w) atomicAdd(dwl + k * HW + e, dz);
+                if (p.w_cpg > 1) atomicAdd(dwl + k * HW + e, dz);
                 else dwl[k * HW + e] = dz;
             }
             // transposed stencil: position q passes w_k a to q + k - 1

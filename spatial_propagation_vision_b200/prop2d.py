@@ -46,6 +46,8 @@ lib.gspn_prop2d_fwd_algo.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 9 + [_vp, _vp]
 lib.gspn_prop2d_fwd_algo.restype = _i
 lib.gspn_prop2d_bwd.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 5
 lib.gspn_prop2d_bwd.restype = _i
+lib.gspn_prop2d_bwd_ex.argtypes = [_vp] * 5 + [_i] * 8 + [_vp] * 5
+lib.gspn_prop2d_bwd_ex.restype = _i
 lib.gspn_prop2d_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
 lib.gspn_prop2d_fwd_noalloc.restype = _i
 lib.gspn_prop2d_workspace_bytes.argtypes = [_i] * 7
@@ -207,6 +209,38 @@ def prop2d_bwd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torc
                                  gy.data_ptr(), B, Cc, H, W, int(dirs), int(share_w), _DT[x.dtype],
                                  g["x"].data_ptr(), g["lam"].data_ptr(), g["wlogit"].data_ptr(),
                                  g["u"].data_ptr(), _stream_handle(stream))
+    if st != 0:
+        raise GspnError(st)
+    return g
+
+
+def prop2d_bwd_ex(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torch.Tensor,
+                  gy: torch.Tensor, dirs: int = 15, gate_dirs: int = 4, w_groups: int | None = None,
+                  stream: torch.cuda.Stream | None = None) -> dict:
+    """Gradients of the sharing variants (gspn_prop2d_bwd_ex), layouts of
+    prop2d_fwd_ex: fp32 tensors {"x", "lam", "wlogit", "u"}; a shared input's
+    gradient sums the gradients of its uses."""
+    B, Cc, H, W = _dims(x)
+    if x.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    G = Cc if w_groups is None else int(w_groups)
+    dev = x.device
+    _check("x", x, (B, Cc, H, W), x.dtype, dev)
+    _check("gy", gy, (B, Cc, H, W), x.dtype, dev)
+    _check("lam", lam, (B, gate_dirs, Cc, H, W), x.dtype, dev)
+    _check("u", u, (B, gate_dirs, Cc, H, W), x.dtype, dev)
+    _check("wlogit", wlogit, (B, 4, G, 3, H, W), x.dtype, dev)
+    g = {"x": torch.empty((B, Cc, H, W), dtype=torch.float32, device=dev),
+         "lam": torch.empty((B, gate_dirs, Cc, H, W), dtype=torch.float32, device=dev),
+         "wlogit": torch.empty((B, 4, G, 3, H, W), dtype=torch.float32, device=dev),
+         "u": torch.empty((B, gate_dirs, Cc, H, W), dtype=torch.float32, device=dev)}
+    with torch.cuda.device(dev):
+        st = lib.gspn_prop2d_bwd_ex(x.data_ptr(), lam.data_ptr(), wlogit.data_ptr(), u.data_ptr(),
+                                    gy.data_ptr(), B, Cc, H, W, int(dirs), int(gate_dirs), G,
+                                    _DT[x.dtype], g["x"].data_ptr(), g["lam"].data_ptr(),
+                                    g["wlogit"].data_ptr(), g["u"].data_ptr(), _stream_handle(stream))
     if st != 0:
         raise GspnError(st)
     return g

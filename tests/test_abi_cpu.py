@@ -153,3 +153,22 @@ def _fwd_algo(lib):
 def test_algo_argument_checks(lib, args, status):
     """gspn_prop2d_fwd_algo rejects bad arguments before it touches a device."""
     assert _fwd_algo(lib)(*args, None) == status
+
+
+def _bwd_ex(lib):
+    f = lib.gspn_prop2d_bwd_ex
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 8 + [ctypes.c_void_p] * 5
+    f.restype = ctypes.c_int
+    return f
+
+
+@pytest.mark.parametrize("args,status", [
+    ((P, P, P, P, P, 1, 4, 8, 8, 15, 2, 4, 0, P, P, P, P), 10),    # gate_dirs neither 1 nor 4
+    ((P, P, P, P, P, 1, 4, 8, 8, 15, 1, 3, 0, P, P, P, P), 10),    # w_groups does not divide Cc
+    ((P, P, P, P, P, 1, 4, 8, 8, 0, 1, 2, 0, P, P, P, P), 3),      # empty direction mask
+    ((P, P, P, P, P, -1, 4, 8, 8, 15, 1, 2, 0, P, P, P, P), 2),    # negative B
+    ((None,) * 5 + (0, 4, 8, 8, 15, 1, 2, 0) + (None,) * 4, 0),     # empty batch
+])
+def test_bwd_ex_argument_checks(lib, args, status):
+    """gspn_prop2d_bwd_ex rejects bad arguments before it touches a device."""
+    assert _bwd_ex(lib)(*args, None) == status

@@ -83,3 +83,35 @@ def test_backward_1k_workload(gspn):
     w = WORKLOADS["1k"]
     rel = check_bwd(gspn, workload_inputs(w, seed=0), seed=9, what="1k")
     print(f"\n1k backward: worst max|err| / max|g| = {rel:.3e}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 4, 16, 20), (2, 6, 37, 38), (1, 4, 74, 74)],
+                         ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("gate_dirs,groups", [(1, "all"), (4, "half"), (1, "one"), (1, "half")])
+def test_backward_sharing_variants(gspn, shape, dtype, gate_dirs, groups):
+    """Gradients of the sharing variants (shared gates sum over the
+    directions, grouped logits over their channels) against the oracle."""
+    B, Cc, H, W = shape
+    G = {"all": Cc, "half": Cc // 2, "one": 1}[groups]
+    g = torch.Generator().manual_seed(hash((shape, gate_dirs, G)) % 2**31)
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x = torch.randn((B, Cc, H, W), generator=g)
+    lam = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
+    wl = torch.randn((B, 4, G, 3, H, W), generator=g) * 2.0
+    u = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
+    gy = torch.randn((B, Cc, H, W), generator=g)
+    inp = {k: v.to(td) for k, v in {"x": x, "lam": lam, "wlogit": wl, "u": u, "gy": gy}.items()}
+    d = {k: v.cuda() for k, v in inp.items()}
+    got = gspn.prop2d_bwd_ex(d["x"], d["lam"], d["wlogit"], d["u"], d["gy"], gate_dirs=gate_dirs,
+                             w_groups=G)
+    torch.cuda.synchronize()
+    assert gspn.launch_info()["path"] == "bwd"
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    want = oracle.prop2d_bwd_ex(f64(inp["x"]), f64(inp["lam"]), f64(inp["wlogit"]), f64(inp["u"]),
+                                f64(inp["gy"]), gate_dirs=gate_dirs, w_groups=G)
+    tol = 1e-4 if dtype == "f32" else 2e-2
+    for k in ("x", "lam", "wlogit", "u"):
+        scale = float(np.max(np.abs(want[k])))
+        err = float(np.max(np.abs(f64(got[k]) - want[k])))
+        assert err <= tol * max(scale, 1e-30), f"{k}: {err:.3e} > {tol} * {scale:.3e}"
