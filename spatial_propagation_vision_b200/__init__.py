@@ -6,11 +6,15 @@ this package does not load the library; ``prop2d`` does, and fails loudly
 when it is missing.
 """
 
-__all__ = ["prop2d_fwd", "workloads"]
+__all__ = ["prop2d_fwd", "prop2d_fwd_ex", "prop2d_bwd", "prop2d_bwd_ex", "prop2d_autograd",
+           "workloads"]
+
+_LAZY = ("prop2d_fwd", "prop2d_fwd_ex", "prop2d_fwd_noalloc", "prop2d_fwd_host",
+         "prop2d_bwd", "prop2d_bwd_ex", "prop2d_autograd", "Prop2DFunction", "launch_info", "lib")
 
 
 def __getattr__(name):
-    if name in ("prop2d_fwd", "prop2d_fwd_host", "lib"):
+    if name in _LAZY:
         from . import prop2d
         return getattr(prop2d, name)
     raise AttributeError(name)

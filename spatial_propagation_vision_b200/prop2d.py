@@ -314,3 +314,31 @@ def launch_info() -> dict:
                               ctypes.byref(path))
     return {"launches": n.value, "grid": g.value, "block": b.value, "smem": s.value,
             "path": (path.value or b"").decode()}
+
+
+class Prop2DFunction(torch.autograd.Function):
+    """Prop2D as an autograd function: the forward is gspn_prop2d_fwd_ex, the
+    backward gspn_prop2d_bwd_ex (the inputs' gradients are computed in fp32
+    and returned in the inputs' dtype)."""
+
+    @staticmethod
+    def forward(ctx, x, lam, wlogit, u, dirs: int = 15, gate_dirs: int = 4, w_groups=None):
+        ctx.save_for_backward(x, lam, wlogit, u)
+        ctx.conf = (int(dirs), int(gate_dirs), w_groups)
+        return prop2d_fwd_ex(x, lam, wlogit, u, dirs=dirs, gate_dirs=gate_dirs, w_groups=w_groups)
+
+    @staticmethod
+    def backward(ctx, gy):
+        x, lam, wlogit, u = ctx.saved_tensors
+        dirs, gate_dirs, w_groups = ctx.conf
+        g = prop2d_bwd_ex(x, lam, wlogit, u, gy.contiguous().to(x.dtype), dirs=dirs,
+                          gate_dirs=gate_dirs, w_groups=w_groups)
+        return (g["x"].to(x.dtype), g["lam"].to(lam.dtype), g["wlogit"].to(wlogit.dtype),
+                g["u"].to(u.dtype), None, None, None)
+
+
+def prop2d_autograd(x: torch.Tensor, lam: torch.Tensor, wlogit: torch.Tensor, u: torch.Tensor,
+                    dirs: int = 15, gate_dirs: int = 4, w_groups: int | None = None) -> torch.Tensor:
+    """y = Prop2D(x; u, lambda, w) with gradients for x, lam, wlogit and u
+    (layouts of prop2d_fwd_ex)."""
+    return Prop2DFunction.apply(x, lam, wlogit, u, dirs, gate_dirs, w_groups)

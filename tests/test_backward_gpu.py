@@ -115,3 +115,27 @@ def test_backward_sharing_variants(gspn, shape, dtype, gate_dirs, groups):
         scale = float(np.max(np.abs(want[k])))
         err = float(np.max(np.abs(f64(got[k]) - want[k])))
         assert err <= tol * max(scale, 1e-30), f"{k}: {err:.3e} > {tol} * {scale:.3e}"
+
+
+@pytest.mark.parametrize("gate_dirs,groups", [(4, "all"), (1, "one")])
+def test_autograd_function(gspn, gate_dirs, groups):
+    """Prop2DFunction: torch autograd through the library's forward and
+    backward matches the oracle's gradients of L = sum(gy * y)."""
+    B, Cc, H, W = 2, 4, 20, 18
+    G = Cc if groups == "all" else 1
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn((B, Cc, H, W), generator=g)
+    lam = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
+    wl = torch.randn((B, 4, G, 3, H, W), generator=g) * 2.0
+    u = torch.rand((B, gate_dirs, Cc, H, W), generator=g)
+    gy = torch.randn((B, Cc, H, W), generator=g)
+    leaves = [t.cuda().requires_grad_() for t in (x, lam, wl, u)]
+    y = gspn.prop2d_autograd(*leaves, gate_dirs=gate_dirs, w_groups=G)
+    (y * gy.cuda()).sum().backward()
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    want = oracle.prop2d_bwd_ex(f64(x), f64(lam), f64(wl), f64(u), f64(gy), gate_dirs=gate_dirs,
+                                w_groups=G)
+    for leaf, k in zip(leaves, ("x", "lam", "wlogit", "u")):
+        scale = float(np.max(np.abs(want[k])))
+        err = float(np.max(np.abs(f64(leaf.grad) - want[k])))
+        assert err <= 1e-4 * max(scale, 1e-30), f"{k}: {err:.3e} vs {scale:.3e}"
