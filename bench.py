@@ -467,6 +467,46 @@ def run_ours(args, w):
     print(json.dumps(line), flush=True)
 
 
+def backward_bytes(w) -> int:
+    """Bytes the backward must move once: x, lambda, u, the logits and gy
+    read (input dtype), the fp32 gradients of x, lambda, u and the logits
+    written."""
+    s = w.in_bytes
+    nd = bin(w.dirs).count("1")
+    E = w.elems
+    logits = 3 * nd * w.B * (1 if w.share_w else w.Cc) * w.H * w.W
+    return E * s * (2 + 2 * nd) + logits * s + 4 * (E * (1 + 2 * nd) + logits)
+
+
+def run_backward(args, w):
+    """`--pass bwd`: gspn_prop2d_bwd on the workload, one GPU (a separate
+    line; the default line is the forward's)."""
+    from spatial_propagation_vision_b200 import prop2d
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    d = {k: v.to(dev) for k, v in workload_inputs(w, seed=0).items()}
+    gy = torch.randn(tuple(d["x"].shape), generator=torch.Generator().manual_seed(1)).to(d["x"].dtype).to(dev)
+    call = lambda: prop2d.prop2d_bwd(d["x"], d["lam"], d["wlogit"], d["u"], gy, dirs=w.dirs,
+                                     share_w=w.share_w)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    nb = backward_bytes(w)
+    print(json.dumps({"metric": "Prop2D bwd GB/s (bytes moved once / time); ms/call", "pass": "bwd",
+                      "value": nb / ms / 1e6, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                      "dtype": {2: "bf16", 4: "f32"}[w.in_bytes], "data": "synthetic (seeded)",
+                      "config": {"workload": w.name, "bytes_per_step": nb},
+                      "launch": prop2d.launch_info()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,6 +521,8 @@ def main():
     ap.add_argument("--cc", type=int, default=None,
                     help="override the workload's channel count (a smaller case of the same "
                          "kernel, for ncu captures that must stay within a few GB)")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd: time gspn_prop2d_bwd on the workload instead (one GPU, own line)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if captured for "
                          "the current build")
@@ -491,7 +533,9 @@ def main():
     if args.cc is not None:
         import dataclasses
         w = dataclasses.replace(w, Cc=args.cc, name=f"{w.name}-cc{args.cc}")
-    if args.impl == "reference":
+    if args.pass_ == "bwd":
+        run_backward(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)
