@@ -78,11 +78,32 @@ def test_backward_clamped(gspn):
     check_bwd(gspn, inp, seed=4, what="clamped")
 
 
-def test_backward_1k_workload(gspn):
-    """The 1k workload's shape (B=32, Cc=64, 74x74, bf16), every plane."""
-    w = WORKLOADS["1k"]
-    rel = check_bwd(gspn, workload_inputs(w, seed=0), seed=9, what="1k")
-    print(f"\n1k backward: worst max|err| / max|g| = {rel:.3e}")
+@pytest.mark.parametrize("name", ["1k", "2k", "mid"])
+def test_backward_workload(gspn, name):
+    """A benchmark workload's shape (1k: B=32, Cc=64, 74x74 bf16; 2k: 8x64x148x148
+    bf16 with logits shared by the channels; mid: 8x64x37x37 fp32), every plane."""
+    w = WORKLOADS[name]
+    rel = check_bwd(gspn, workload_inputs(w, seed=0), share_w=w.share_w, seed=9, what=name)
+    print(f"\n{name} backward: worst max|err| / max|g| = {rel:.3e}")
+
+
+@pytest.mark.parametrize("dtype,shape", [("f32", (1, 2, 19, 23)), ("bf16", (2, 3, 74, 74)),
+                                         ("f32", (1, 1, 100, 130))],
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_backward_nan_in_off_grid_slots(gspn, dtype, shape):
+    """Off-grid logit slots (slot 0 of a line's first position, slot 2 of its
+    last) carry no weight; filled with NaN they must reach no gradient, and
+    their own gradient is zero (the oracle never reads them)."""
+    B, Cc, H, W = shape
+    inp = make_inputs(B, Cc, H, W, sigma_w=2.0, dtype=dtype, seed=23)
+    wl = inp["wlogit"].clone()
+    nan = float("nan")
+    wl[:, 0:2, :, 0, :, 0] = nan
+    wl[:, 0:2, :, 2, :, W - 1] = nan
+    wl[:, 2:4, :, 0, 0, :] = nan
+    wl[:, 2:4, :, 2, H - 1, :] = nan
+    inp["wlogit"] = wl
+    check_bwd(gspn, inp, seed=5, what=f"NaN edge slots {shape} {dtype}")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
