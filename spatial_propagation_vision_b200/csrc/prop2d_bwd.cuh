@@ -124,10 +124,11 @@ struct BwdLine {
         }
     }
 
-    // normalised weights (w), sigmoids (s) and local sum (S) of position
-    // q = lane R + r; off-grid slots are selected away
+    // normalised weights (w), sigmoids (s), local sum (S) and the
+    // reciprocal of the clamped sum (rs = 1 / max(S, eps), hardware
+    // reciprocal) of position q = lane R + r; off-grid slots are selected away
     __device__ __forceinline__ void weights(const BwdIn<R> &in, int r, int q, float (&s)[3], float (&w)[3],
-                                            float &S) const {
+                                            float &S, float &rs) const {
         S = 0.f;
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
@@ -135,7 +136,7 @@ struct BwdLine {
             s[k] = (nb >= 0 && nb < M) ? bwd_sigmoid(in.z[k][r]) : 0.f;
             S += s[k];
         }
-        const float rs = 1.0f / fmaxf(S, 1e-6f);
+        rs = rcp(fmaxf(S, 1e-6f));
 #pragma unroll
         for (int k = 0; k < 3; ++k) w[k] = s[k] * rs;
     }
@@ -149,8 +150,8 @@ struct BwdLine {
         for (int r = 0; r < R; ++r) {
             const int q = lane * R + r;
             if (q >= M) { hn[r] = 0.f; continue; }
-            float sg[3], w[3], S;
-            weights(in, r, q, sg, w, S);
+            float sg[3], w[3], S, rs;
+            weights(in, r, q, sg, w, S, rs);
             const float left = r > 0 ? h[r > 0 ? r - 1 : 0] : (lane > 0 ? hl : 0.f);
             const float right = r + 1 < R ? h[r + 1 < R ? r + 1 : r] : hr;
             hn[r] = w[0] * left + w[1] * h[r] + w[2] * right + in.lam[r] * in.x[r];
@@ -212,8 +213,8 @@ struct BwdLine {
                 dlam[e] = a * in.x[r];
             }
             atomicAdd(dx + e, a * in.lam[r]);
-            float sgm[3], w[3], S;
-            weights(in, r, q, sgm, w, S);
+            float sgm[3], w[3], S, rs;
+            weights(in, r, q, sgm, w, S, rs);
             float dw[3], dot = 0.f;
 #pragma unroll
             for (int k = 0; k < 3; ++k) {
@@ -225,7 +226,8 @@ struct BwdLine {
             for (int k = 0; k < 3; ++k) {
                 const int nb = q + k - 1;
                 if (nb < 0 || nb >= M) continue;
-                const float ds = S > 1e-6f ? (dw[k] - dot) / S : dw[k] * 1e6f;
+                // (dw_j - sum_k dw_k w_k) / S, or dw_j / eps where the clamp holds
+                const float ds = (S > 1e-6f ? dw[k] - dot : dw[k]) * rs;
                 const float dz = ds * sgm[k] * (1.f - sgm[k]);
                 if (p.w_cpg > 1) atomicAdd(dwl + k * HW + e, dz);
                 else dwl[k * HW + e] = dz;
