@@ -24,7 +24,7 @@
 // Weights are recomputed in the plain form (sigmoid, local sum, clamp,
 // divide) in fp32 in both sweeps.  Every sweep loads the next line's inputs
 // one step ahead, into registers, so that a step does not wait for its own
-// loads.  Gradients are fp32: dlambda, du and (per
+// loads (two lines ahead measured slower).  Gradients are fp32: dlambda, du and (per
 // channel) dwlogit are stored once; dx adds the four directions with global
 // fp32 atomics, and shared inputs add over their uses likewise (lambda and u
 // shared by the four directions: their gradients add over the directions;
@@ -77,12 +77,18 @@ struct BwdLine {
     const int lane, d;
     const bool fwd, rows;
     const int L, M;
-    const T *x, *lam, *u, *gy, *wl;   // this plane's tensors (direction d)
-    float *dx, *dlam, *du, *dwl;
+    const int lstride;                 // elements between consecutive lines: W (rows) or 1 (columns)
+    const bool gate_shared, w_shared;  // lambda/u shared by the directions; logits by channels
+    int qo_[R];           // element offset of position lane R + r within a line (clamped to M - 1)
+    bool valid_[R];       // lane R + r < M
+    bool on0_[R], on2_[R];    // the slot k = 0 / k = 2 neighbour is on the line (valid positions)
+    const T *x, *lam, *u, *gy, *wl0, *wl1, *wl2;   // this plane's tensors (direction d)
+    float *dx, *dlam, *du, *dwl0, *dwl1, *dwl2;
 
     __device__ BwdLine(const BwdParams &p_, int lane_, int d_, int b, int c)
         : p(p_), lane(lane_), d(d_), fwd((d_ & 1) == 0), rows(d_ < 2),
-          L(d_ < 2 ? p_.H : p_.W), M(d_ < 2 ? p_.W : p_.H) {
+          L(d_ < 2 ? p_.H : p_.W), M(d_ < 2 ? p_.W : p_.H), lstride(d_ < 2 ? p_.W : 1),
+          gate_shared(p_.gate_dirs == 1), w_shared(p_.w_cpg > 1) {
         const size_t HW = static_cast<size_t>(p.H) * p.W;
         const size_t xo = (static_cast<size_t>(b) * p.Cc + c) * HW;
         const size_t go = ((static_cast<size_t>(b) * p.gate_dirs + (p.gate_dirs == 4 ? d : 0)) * p.Cc + c) * HW;
@@ -91,30 +97,45 @@ struct BwdLine {
         gy = static_cast<const T *>(p.gy) + xo;
         lam = static_cast<const T *>(p.lam) + go;
         u = static_cast<const T *>(p.u) + go;
-        wl = static_cast<const T *>(p.wl) + wo;
+        wl0 = static_cast<const T *>(p.wl) + wo;
+        wl1 = wl0 + HW;
+        wl2 = wl1 + HW;
         dx = p.dx + xo;
         dlam = p.dlam + go;
         du = p.du + go;
-        dwl = p.dwl + wo;
+        dwl0 = p.dwl + wo;
+        dwl1 = dwl0 + HW;
+        dwl2 = dwl1 + HW;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = lane * R + r;
+            const int qc = min(q, M - 1);
+            qo_[r] = rows ? qc : qc * p.W;
+            valid_[r] = q < M;
+            on0_[r] = q < M && q > 0;
+            on2_[r] = q + 1 < M;
+        }
     }
+    __device__ __forceinline__ int qo(int r) const { return qo_[r]; }
+    __device__ __forceinline__ bool valid(int r) const { return valid_[r]; }
+    __device__ __forceinline__ bool on0(int r) const { return on0_[r]; }
+    __device__ __forceinline__ bool on2(int r) const { return on2_[r]; }
 
-    // element index of position q of scan step s within a plane
-    __device__ __forceinline__ size_t idx(int s, int q) const {
-        const int line = fwd ? s : L - 1 - s;
-        return rows ? static_cast<size_t>(line) * p.W + q : static_cast<size_t>(q) * p.W + line;
-    }
+    // element offset of scan line s's first position within the plane
+    // (plane offsets fit 32 bits: H W <= 2^30)
+    __device__ __forceinline__ int loff(int s) const { return (fwd ? s : L - 1 - s) * lstride; }
 
     // Inputs of line s (positions past the line's end read position M-1:
     // finite, never used; off-grid logit slots are read but never used).
     template <bool REV>
     __device__ __forceinline__ void load_in(int s, BwdIn<R> &in) const {
-        const size_t HW = static_cast<size_t>(p.H) * p.W;
+        const int lo = loff(s);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int q = min(lane * R + r, M - 1);
-            const size_t e = idx(s, q);
-#pragma unroll
-            for (int k = 0; k < 3; ++k) in.z[k][r] = bwd_in(wl, k * HW + e);
+            const int e = lo + qo(r);
+            in.z[0][r] = bwd_in(wl0, e);
+            in.z[1][r] = bwd_in(wl1, e);
+            in.z[2][r] = bwd_in(wl2, e);
             in.lam[r] = bwd_in(lam, e);
             in.x[r] = bwd_in(x, e);
             if (REV) {
@@ -126,16 +147,13 @@ struct BwdLine {
 
     // normalised weights (w), sigmoids (s), local sum (S) and the
     // reciprocal of the clamped sum (rs = 1 / max(S, eps), hardware
-    // reciprocal) of position q = lane R + r; off-grid slots are selected away
-    __device__ __forceinline__ void weights(const BwdIn<R> &in, int r, int q, float (&s)[3], float (&w)[3],
+    // reciprocal) of the lane's position r; off-grid slots are selected away
+    __device__ __forceinline__ void weights(const BwdIn<R> &in, int r, float (&s)[3], float (&w)[3],
                                             float &S, float &rs) const {
-        S = 0.f;
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int nb = q + k - 1;
-            s[k] = (nb >= 0 && nb < M) ? bwd_sigmoid(in.z[k][r]) : 0.f;
-            S += s[k];
-        }
+        s[0] = on0(r) ? bwd_sigmoid(in.z[0][r]) : 0.f;
+        s[1] = valid(r) ? bwd_sigmoid(in.z[1][r]) : 0.f;
+        s[2] = on2(r) ? bwd_sigmoid(in.z[2][r]) : 0.f;
+        S = (s[0] + s[1]) + s[2];
         rs = rcp(fmaxf(S, 1e-6f));
 #pragma unroll
         for (int k = 0; k < 3; ++k) w[k] = s[k] * rs;
@@ -148,20 +166,19 @@ struct BwdLine {
         float hn[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int q = lane * R + r;
-            if (q >= M) { hn[r] = 0.f; continue; }
             float sg[3], w[3], S, rs;
-            weights(in, r, q, sg, w, S, rs);
+            weights(in, r, sg, w, S, rs);
             const float left = r > 0 ? h[r > 0 ? r - 1 : 0] : (lane > 0 ? hl : 0.f);
             const float right = r + 1 < R ? h[r + 1 < R ? r + 1 : r] : hr;
-            hn[r] = w[0] * left + w[1] * h[r] + w[2] * right + in.lam[r] * in.x[r];
+            const float v = w[0] * left + w[1] * h[r] + w[2] * right + in.lam[r] * in.x[r];
+            hn[r] = valid(r) ? v : 0.f;
         }
 #pragma unroll
         for (int r = 0; r < R; ++r) h[r] = hn[r];
     }
 
     // steps [s0, s1) forwards from h, storing h after step s into
-    // out(s) when out is given; the next line's inputs load one step ahead
+    // out(s); the next line's inputs load one step ahead
     template <typename Out>
     __device__ __forceinline__ void sweep(int s0, int s1, float (&h)[R], Out out) const {
         BwdIn<R> a, b;
@@ -170,11 +187,10 @@ struct BwdLine {
             if (s + 1 < s1) load_in<false>(s + 1, b);
             fwd_step(a, h);
             out(s, h);
-            if (s + 1 < s1) {
-                if (s + 2 < s1) load_in<false>(s + 2, a);
-                fwd_step(b, h);
-                out(s + 1, h);
-            }
+            if (s + 1 >= s1) break;
+            if (s + 2 < s1) load_in<false>(s + 2, a);
+            fwd_step(b, h);
+            out(s + 1, h);
         }
     }
 
@@ -187,50 +203,57 @@ struct BwdLine {
         for (int r = 0; r < R; ++r) h[r] = buf[lane * R + r];
     }
 
-    // The whole backward of this direction.  `ck`: checkpoint lines
-    // (line i holds h after step i * kSeg + kSeg - 1), `seg`: kSeg + 1 lines
-    // (line 0: h before the segment, line 1 + t: after its step t).
     // The reverse step s (adjoint of line s): gradients of line s's inputs,
     // the carry into line s-1.  hcur / hprv: h after steps s and s-1.
     __device__ __forceinline__ void rev_step(int s, const BwdIn<R> &in, const float *hcur, const float *hprv,
                                              float (&carry)[R]) const {
-        const size_t HW = static_cast<size_t>(p.H) * p.W;
+        const int lo = loff(s);
         float cl = 0.f, cr = 0.f, cmid[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) cmid[r] = 0.f;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int q = lane * R + r;
-            if (q >= M) continue;
-            const size_t e = idx(s, q);
+            const int e = lo + qo(r);
             const float gyv = in.gy[r];
-            const float a = in.u[r] * gyv + carry[r];
-            if (p.gate_dirs == 1) {
-                atomicAdd(du + e, gyv * hcur[q]);
-                atomicAdd(dlam + e, a * in.x[r]);
-            } else {
-                du[e] = gyv * hcur[q];
-                dlam[e] = a * in.x[r];
+            // positions past the line's end take no adjoint: they pass nothing on
+            const float a = valid(r) ? in.u[r] * gyv + carry[r] : 0.f;
+            if (valid(r)) {
+                if (gate_shared) {
+                    atomicAdd(du + e, gyv * hcur[q]);
+                    atomicAdd(dlam + e, a * in.x[r]);
+                } else {
+                    du[e] = gyv * hcur[q];
+                    dlam[e] = a * in.x[r];
+                }
+                atomicAdd(dx + e, a * in.lam[r]);
             }
-            atomicAdd(dx + e, a * in.lam[r]);
             float sgm[3], w[3], S, rs;
-            weights(in, r, q, sgm, w, S, rs);
+            weights(in, r, sgm, w, S, rs);
+            // dw_k = a h_{s-1}(q + k - 1) for on-grid slots (line 0 has no predecessor)
+            float hp[3] = {0.f, 0.f, 0.f};
+            if (s > 0) {
+                if (on0(r)) hp[0] = hprv[q - 1 >= 0 ? q - 1 : 0];
+                if (valid(r)) hp[1] = hprv[q];
+                if (on2(r)) hp[2] = hprv[q + 1];
+            }
             float dw[3], dot = 0.f;
 #pragma unroll
             for (int k = 0; k < 3; ++k) {
-                const int nb = q + k - 1;
-                dw[k] = (nb >= 0 && nb < M && s > 0) ? a * hprv[nb] : 0.f;
+                dw[k] = a * hp[k];
                 dot += dw[k] * w[k];
             }
+            const bool on[3] = {on0(r), valid(r), on2(r)};
+            float *const dwk[3] = {dwl0, dwl1, dwl2};
 #pragma unroll
             for (int k = 0; k < 3; ++k) {
-                const int nb = q + k - 1;
-                if (nb < 0 || nb >= M) continue;
                 // (dw_j - sum_k dw_k w_k) / S, or dw_j / eps where the clamp holds
                 const float ds = (S > 1e-6f ? dw[k] - dot : dw[k]) * rs;
                 const float dz = ds * sgm[k] * (1.f - sgm[k]);
-                if (p.w_cpg > 1) atomicAdd(dwl + k * HW + e, dz);
-                else dwl[k * HW + e] = dz;
+                if (on[k]) {
+                    if (w_shared) atomicAdd(dwk[k] + e, dz);
+                    else dwk[k][e] = dz;
+                }
             }
             // transposed stencil: position q passes w_k a to q + k - 1
             const float c0 = w[0] * a, c1 = w[1] * a, c2 = w[2] * a;
@@ -285,10 +308,9 @@ struct BwdLine {
             for (int s = s1 - 1; s >= s0; s -= 2) {
                 if (s - 1 >= s0) load_in<true>(s - 1, b);
                 rev_step(s, a, seg + (s - s0 + 1) * line_f, seg + (s - s0) * line_f, carry);
-                if (s - 1 >= s0) {
-                    if (s - 2 >= s0) load_in<true>(s - 2, a);
-                    rev_step(s - 1, b, seg + (s - s0) * line_f, seg + (s - 1 - s0) * line_f, carry);
-                }
+                if (s - 1 < s0) break;
+                if (s - 2 >= s0) load_in<true>(s - 2, a);
+                rev_step(s - 1, b, seg + (s - s0) * line_f, seg + (s - 1 - s0) * line_f, carry);
             }
             __syncwarp();
         }
