@@ -106,7 +106,9 @@ bool plan_dir_fit(DirPlan &pl, int cap, int H, int W, int dirs, int mode) {
     // column is a dummy written by row lanes past the end of a row
     const int YP = (W % 2 == 0) ? W + 1 : W + 2;
     const int stage_col = round_up(H * gspn::kColPitch, 16);
-    const int col_ring = gspn::kColStages * stage_col;
+    // global accumulation (fp32 only) stages a chunk's column outputs after
+    // each column ring: (H x 4 + 32) floats (rows shifted one word per lane block)
+    const int col_ring = gspn::kColStages * stage_col + (mode == 1 ? round_up((H * 4 + 32) * 4, 16) : 0);
     const int rings = n_col * col_ring + gspn::kDirBarBytes;
     const int n_planes = mode == 3 ? 1 : ((dirs & 3) ? 1 : 0) + ((dirs & 12) ? 1 : 0);
     // a plane holds its rows plus one dummy row (written by the column lanes

@@ -742,6 +742,21 @@ struct ColScan {
         }
     }
 
+    // fp32 lines of more than 160 positions read one column per step
+    // straight from the stage: two two-column word sets of six or more
+    // positions per lane would hold 144+ registers and spill.
+    static constexpr bool kDirect = es == 4 && R >= 6;
+
+    // fp32: column kk (0..3 in scan order within a strip row) of a stage.
+    __device__ __forceinline__ void load_col(const unsigned char *sp, int kk, float (&v)[kTensors][R]) const {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int off = rowq[r] + 4 * kk;
+#pragma unroll
+            for (int t = 0; t < kTensors; ++t) v[t][r] = *reinterpret_cast<const float *>(sp + off + 16 * t);
+        }
+    }
+
     // bf16: both word sets of body b (columns 4b..4b+3 in scan order) of a
     // stage, one 8-byte read per tensor and position.
     __device__ __forceinline__ void load_quad(const unsigned char *sp, int b, PairSet &A, PairSet &B) const {
@@ -802,6 +817,44 @@ struct ColScan {
         }
     }
 
+    // kYGlobal: the outputs of a chunk's CH columns are staged in shared
+    // memory, [grid row][CH] fp32 in column order after the column ring,
+    // row q at q CH + q / R (one word more per lane block, so that the
+    // lanes' stores of a step fall on distinct banks), and added to the
+    // output once per chunk: a row's CH columns in one 16-byte vector atomic
+    // instead of CH scattered 4-byte ones.
+    __device__ __forceinline__ float *ystage() const { return reinterpret_cast<float *>(ring + NS * p.stage_col); }
+
+    // column j (column order within the chunk) of the step's outputs
+    __device__ __forceinline__ void emit_stage(const float (&h)[R], const LineW<R> &W, int j) const {
+        float *st = ystage();
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int q = lane * R + r;
+            if (g.valid[r]) st[q * CH + j + lane] = W.uu[r] * h[r];
+        }
+    }
+
+    // add the staged outputs of chunk c (n columns scanned) to the output
+    __device__ __forceinline__ void flush_stage(int c, int n, float *yg) const {
+        __syncwarp();
+        const float *st = ystage();
+        const int lo = chunk_lo(c);
+        // a full chunk on a 16-byte boundary: one vector atomic per row
+        const bool vec = CH == 4 && n == CH && lo >= 0 && lo % 4 == 0 && p.W % 4 == 0;
+        const int j0 = fwd ? 0 : CH - n;   // the chunk's scanned columns: j0 .. j0 + n - 1
+        for (int i = lane; i < p.H; i += 32) {
+            const float *sr = st + i * CH + i / R;
+            float *o = yg + static_cast<size_t>(i) * p.W + lo;
+            if (vec) {
+                atomicAdd(reinterpret_cast<float4 *>(o), make_float4(sr[0], sr[1], sr[2], sr[3]));
+            } else {
+                for (int j = j0; j < j0 + n; ++j) atomicAdd(o + j, sr[j]);
+            }
+        }
+        __syncwarp();
+    }
+
     __device__ __forceinline__ void emit(const float (&h)[R], const LineW<R> &W, int col, float *ys,
                                          float *yg, bool first) const {
         const int yc = ycol(col);
@@ -837,13 +890,29 @@ struct ColScan {
         // weights of the next step (when none follows: stale but finite
         // words, never used)
         float v[kTensors][R];
-        if (J == 0) unpack<1>(A, v);
-        else if (J == 1) unpack<0>(B, v);
-        else if (J == 2) unpack<1>(B, v);
-        else unpack<0>(A, v);
+        if constexpr (kDirect) {
+            // the next step's column, read from the stage now
+            if (J < 3) {
+                load_col(stage_ptr(gi), J + 1, v);
+            } else if (more) {
+                wait<0>();               // chunk gi+1 (issued when chunk gi was entered)
+                load_col(stage_ptr(gi + 1), 0, v);
+            } else {
+                load_col(stage_ptr(gi), 3, v);
+            }
+        } else if (J == 0) {
+            unpack<1>(A, v);
+        } else if (J == 1) {
+            unpack<0>(B, v);
+        } else if (J == 2) {
+            unpack<1>(B, v);
+        } else {
+            unpack<0>(A, v);
+        }
         // word sets of the steps ahead, read after the step's last use of
         // the set they replace
-        if constexpr (es == 2) {
+        if constexpr (kDirect) {
+        } else if constexpr (es == 2) {
             if (J == 2 && more) {
                 if (b + 1 < NB) {
                     load_quad(stage_ptr(gi), b + 1, A, B);
@@ -865,6 +934,7 @@ struct ColScan {
         }
         const bool bad = next_weights<PRE>(v, g, Wb[(J + 1) & 1]);
         if constexpr (MODE == kYHalf) emit_half<J>(h, Wc, fwd ? st : L - 1 - st, ys, st < split);
+        else if constexpr (MODE == kYGlobal) emit_stage(h, Wc, fwd ? k : CH - 1 - k);
         else emit(h, Wc, fwd ? st : L - 1 - st, ys, yg, st < split);
         if (!PRE) line_terms_fix(bad, v, g, Wb[(J + 1) & 1]);
         if (MODE != kYGlobal && MODE != kYShared && st + 1 == split) pair_barrier(3);
@@ -892,9 +962,13 @@ struct ColScan {
                 // the item's first chunk: wait for it, weights of step 0
                 wait<1>();
                 float v[kTensors][R];
-                if constexpr (es == 2) load_quad(stage_ptr(gi), 0, A, B);
-                else load_pair(stage_ptr(gi), 0, A);
-                unpack<0>(A, v);
+                if constexpr (kDirect) {
+                    load_col(stage_ptr(gi), 0, v);
+                } else {
+                    if constexpr (es == 2) load_quad(stage_ptr(gi), 0, A, B);
+                    else load_pair(stage_ptr(gi), 0, A);
+                    unpack<0>(A, v);
+                }
                 first_weights<PRE>(v, g, Wb[0]);
             }
             const bool last = c + 1 == nch;
@@ -906,6 +980,7 @@ struct ColScan {
                 bstep<2>(gi, c, b, last, n, h, Wb, A, B, ys, yg);
                 bstep<3>(gi, c, b, last, n, h, Wb, A, B, ys, yg);
             }
+            if constexpr (MODE == kYGlobal) flush_stage(c, n, yg);
         }
     }
 };

@@ -362,6 +362,8 @@ def test_nan_in_off_grid_slots(gspn, dtype, shape, path):
     ((8, 40, 20, 33), "bf16", "generic"),      # odd bf16 row width
     ((1, 2, 160, 160), "f32", "dir-shared"),   # lines over 128; two output planes do not fit
     ((1, 2, 256, 256), "f32", "dir-yglobal"),
+    ((1, 1, 256, 250), "f32", "dir-yglobal"),   # width not a multiple of 4: scalar column flush
+    ((1, 1, 231, 253), "f32", "dir-yglobal"),   # odd width: a last column chunk of one column
     ((1, 2, 256, 256), "bf16", "dir-banded"),
     ((1, 2, 148, 148), "bf16", "dir-half"),
     ((1, 1, 300, 40), "f32", "generic"),       # line longer than 256
